@@ -1,0 +1,278 @@
+"""Block-sparse masked attention forward for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding of the C ABI in ``include/fa_b200.h``.  It only marshals arguments:
+every step of the computation runs in the library's CUDA kernels.  PyTorch supplies device
+memory and streams.  There is no CPU fallback: importing this package fails loudly if the
+shared library has not been built (``python -m block_sparse_masked_x128_b200.build``).
+
+Low-level names mirror the C entry points (``fa_create_block_mask``, ``fa_forward``, ...).
+``create_block_mask`` and ``flex_attention`` are the convenience forms named after the
+FlexAttention API the pages use ("How to Use FlexAttention on Apple Silicon", Setup).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libfa_b200.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with `python -m block_sparse_masked_x128_b200.build`")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+# ---------------------------------------------------------------- constants (fa_b200.h)
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_CUDA = 3
+FA_ERR_OOM = 4
+FA_ERR_TIMEOUT = 5
+FA_ERR_INTERNAL = 6
+
+FA_MASK_CAUSAL = 1
+FA_MASK_SLIDING_WINDOW = 2
+FA_MASK_DOCUMENT = 4
+FA_SCORE_NONE = 0
+FA_SCORE_SOFTCAP = 1
+FA_SCORE_ALIBI = 2
+FA_DTYPE_F16 = 0
+FA_DTYPE_BF16 = 1
+
+EXPORTED = ("fa_create_block_mask", "fa_forward", "fa_block_mask_get", "fa_get_device_status",
+            "fa_destroy_block_mask", "fa_status_string", "fa_last_error_message")
+
+
+class FaMaskParams(ctypes.Structure):
+    _fields_ = [("window", ctypes.c_int32), ("doc_id", ctypes.c_void_p),
+                ("separate_full_blocks", ctypes.c_int32)]
+
+
+class FaScoreParams(ctypes.Structure):
+    _fields_ = [("softcap", ctypes.c_float), ("alibi_slopes", ctypes.c_void_p)]
+
+
+class FaTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32),
+                ("B", ctypes.c_int64), ("H", ctypes.c_int64), ("S", ctypes.c_int64),
+                ("D", ctypes.c_int64), ("stride", ctypes.c_int64 * 4)]
+
+
+class FaBlockMaskInfo(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("Q_LEN", ctypes.c_int32),
+                ("KV_LEN", ctypes.c_int32), ("BLOCK_SIZE", ctypes.c_int32),
+                ("q_blocks", ctypes.c_int32), ("kv_blocks", ctypes.c_int32),
+                ("mask_kind", ctypes.c_uint32), ("window", ctypes.c_int32),
+                ("separate_full_blocks", ctypes.c_int32),
+                ("kv_num_blocks", ctypes.c_void_p), ("kv_indices", ctypes.c_void_p),
+                ("full_kv_num_blocks", ctypes.c_void_p), ("full_kv_indices", ctypes.c_void_p)]
+
+
+_status = ctypes.c_int
+_lib.fa_create_block_mask.argtypes = [ctypes.c_uint32, ctypes.POINTER(FaMaskParams), ctypes.c_int32,
+                                      ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p)]
+_lib.fa_create_block_mask.restype = _status
+_lib.fa_forward.argtypes = [ctypes.POINTER(FaTensor), ctypes.POINTER(FaTensor), ctypes.POINTER(FaTensor),
+                            ctypes.c_void_p, ctypes.c_uint32, ctypes.POINTER(FaScoreParams),
+                            ctypes.c_float, ctypes.POINTER(FaTensor), ctypes.c_void_p, ctypes.c_void_p]
+_lib.fa_forward.restype = _status
+_lib.fa_block_mask_get.argtypes = [ctypes.c_void_p, ctypes.POINTER(FaBlockMaskInfo)]
+_lib.fa_block_mask_get.restype = _status
+_lib.fa_get_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+_lib.fa_get_device_status.restype = _status
+_lib.fa_destroy_block_mask.argtypes = [ctypes.c_void_p]
+_lib.fa_destroy_block_mask.restype = None
+_lib.fa_status_string.argtypes = [ctypes.c_int]
+_lib.fa_status_string.restype = ctypes.c_char_p
+_lib.fa_last_error_message.argtypes = []
+_lib.fa_last_error_message.restype = ctypes.c_char_p
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.fa_last_error_message().decode()
+        super().__init__(f"{where}: {_lib.fa_status_string(status).decode()}: {msg}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != FA_OK:
+        raise FaError(status, where)
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def fa_status_string(status: int) -> str:
+    return _lib.fa_status_string(status).decode()
+
+
+def fa_last_error_message() -> str:
+    return _lib.fa_last_error_message().decode()
+
+
+# ---------------------------------------------------------------- low-level entry points
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _dtype_code(dtype) -> int:
+    import torch
+    if dtype == torch.bfloat16:
+        return FA_DTYPE_BF16
+    if dtype == torch.float16:
+        return FA_DTYPE_F16
+    raise TypeError(f"unsupported dtype {dtype}: use torch.float16 or torch.bfloat16")
+
+
+def fa_tensor(t) -> FaTensor:
+    """Describe a 4-D (B, H, S, D) torch tensor for the C ABI (no copy)."""
+    if t.dim() != 4:
+        raise ValueError("expected a (B, H, S, D) tensor")
+    st = (ctypes.c_int64 * 4)(*t.stride())
+    B, H, S, D = t.shape
+    return FaTensor(t.data_ptr(), _dtype_code(t.dtype), B, H, S, D, st)
+
+
+def fa_create_block_mask(mask_kind: int, params: Optional[FaMaskParams], B: int, H: int,
+                         Q_LEN: int, KV_LEN: int, BLOCK_SIZE: int = 128, stream=None) -> int:
+    """Call fa_create_block_mask; returns the raw handle (raises FaError on failure)."""
+    h = ctypes.c_void_p()
+    st = _lib.fa_create_block_mask(mask_kind, ctypes.byref(params) if params is not None else None,
+                                   B, H, Q_LEN, KV_LEN, BLOCK_SIZE, _stream_ptr(stream), ctypes.byref(h))
+    _check(st, "fa_create_block_mask")
+    return h.value
+
+
+def fa_forward(q: FaTensor, k: FaTensor, v: FaTensor, block_mask: int, score_mod_kind: int,
+               params: Optional[FaScoreParams], scale: float, out: FaTensor, lse_ptr: Optional[int],
+               stream=None) -> None:
+    st = _lib.fa_forward(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), block_mask, score_mod_kind,
+                         ctypes.byref(params) if params is not None else None, scale, ctypes.byref(out),
+                         lse_ptr, _stream_ptr(stream))
+    _check(st, "fa_forward")
+
+
+def fa_block_mask_get(block_mask: int) -> FaBlockMaskInfo:
+    info = FaBlockMaskInfo()
+    _check(_lib.fa_block_mask_get(block_mask, ctypes.byref(info)), "fa_block_mask_get")
+    return info
+
+
+def fa_get_device_status(block_mask: int, stream=None) -> int:
+    """Synchronise the stream and return the status code (FA_OK or FA_ERR_TIMEOUT ...)."""
+    return _lib.fa_get_device_status(block_mask, _stream_ptr(stream))
+
+
+def fa_destroy_block_mask(block_mask: int) -> None:
+    _lib.fa_destroy_block_mask(block_mask)
+
+
+# ---------------------------------------------------------------- convenience API
+
+class _DeviceArray:
+    """Zero-copy view of library-owned int32 device memory (for torch.as_tensor)."""
+
+    def __init__(self, ptr: int, shape):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": "<i4",
+                                         "data": (ptr, True), "version": 3, "strides": None}
+
+
+class BlockMask:
+    """A block mask built on the GPU; release happens when the object is collected.
+
+    Attributes ``kv_num_blocks``, ``kv_indices``, ``full_kv_num_blocks`` and
+    ``full_kv_indices`` are int32 CUDA tensors copied out of the library's buffers.
+    """
+
+    def __init__(self, handle: int, device, keepalive=None):
+        self.handle = handle
+        self.device = device
+        self._keepalive = keepalive
+        self.info = fa_block_mask_get(handle)
+
+    def _view(self, ptr, shape):
+        import torch
+        return torch.as_tensor(_DeviceArray(ptr, shape), device=self.device).clone()
+
+    @property
+    def shape_prefix(self):
+        return (self.info.B, self.info.H, self.info.q_blocks)
+
+    @property
+    def kv_num_blocks(self):
+        return self._view(self.info.kv_num_blocks, self.shape_prefix)
+
+    @property
+    def kv_indices(self):
+        return self._view(self.info.kv_indices, self.shape_prefix + (self.info.kv_blocks,))
+
+    @property
+    def full_kv_num_blocks(self):
+        return self._view(self.info.full_kv_num_blocks, self.shape_prefix)
+
+    @property
+    def full_kv_indices(self):
+        return self._view(self.info.full_kv_indices, self.shape_prefix + (self.info.kv_blocks,))
+
+    def device_status(self, stream=None) -> int:
+        return fa_get_device_status(self.handle, stream)
+
+    def __del__(self):
+        h, self.handle = getattr(self, "handle", None), None
+        if h:
+            try:
+                fa_destroy_block_mask(h)
+            except Exception:
+                pass
+
+
+def create_block_mask(mask_kind: int, B: Optional[int], H: Optional[int], Q_LEN: int, KV_LEN: int,
+                      *, window: int = 0, doc_id=None, separate_full_blocks: bool = True,
+                      BLOCK_SIZE: int = 128, device=None, stream=None) -> BlockMask:
+    """Build a block mask on the current CUDA device (B or H of None broadcasts)."""
+    import torch
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    doc_ptr = None
+    if doc_id is not None:
+        if not (doc_id.is_cuda and doc_id.dtype == torch.int32 and doc_id.is_contiguous()):
+            raise ValueError("doc_id must be a contiguous int32 CUDA tensor")
+        doc_ptr = doc_id.data_ptr()
+    params = FaMaskParams(int(window), doc_ptr, 1 if separate_full_blocks else 0)
+    with torch.cuda.device(dev):
+        h = fa_create_block_mask(int(mask_kind), params, int(B or 0), int(H or 0), int(Q_LEN),
+                                 int(KV_LEN), int(BLOCK_SIZE), stream)
+    # doc_id is copied on the stream; keep it alive until the caller's stream has run it.
+    return BlockMask(h, dev, keepalive=doc_id)
+
+
+def flex_attention(q, k, v, block_mask: BlockMask, *, score_mod: int = FA_SCORE_NONE,
+                   softcap: float = 30.0, alibi_slopes=None, scale: Optional[float] = None,
+                   out=None, lse=None, return_lse: bool = True, stream=None) -> Tuple:
+    """Fused block-sparse attention forward: returns (out, lse) (lse None if not requested)."""
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty(q.shape[0], q.shape[1], q.shape[2], device=q.device, dtype=torch.float32)
+    slopes_ptr = None
+    if alibi_slopes is not None:
+        if not (alibi_slopes.is_cuda and alibi_slopes.dtype == torch.float32):
+            raise ValueError("alibi_slopes must be a float32 CUDA tensor")
+        slopes_ptr = alibi_slopes.data_ptr()
+    params = FaScoreParams(float(softcap), slopes_ptr)
+    fa_forward(fa_tensor(q), fa_tensor(k), fa_tensor(v), block_mask.handle, int(score_mod), params,
+               float(scale) if scale is not None else -1.0, fa_tensor(out),
+               lse.data_ptr() if lse is not None else None, stream)
+    return out, lse
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

@@ -1,0 +1,615 @@
+// attn_fwd.cu -- fused block-sparse attention forward for sm_100a.
+//
+// What it computes ("How to Use FlexAttention on Apple Silicon", "The two hooks" and
+// "Bonus: a score_mod for soft-capping"):
+//   O = softmax(mask(score_mod(scale * Q K^T))) V,  lse = log-sum-exp per query row,
+// visiting only the tiles a block mask lists, evaluating the mask only on partial
+// tiles and never writing the score matrix to memory.
+//
+// Organisation (one persistent CTA per SM, 12 warps):
+//   warp 0      TMA producer: Q tiles of the unit, then K_j, V_j of every listed kv block
+//               into a ring of shared-memory stages (128-byte swizzle).
+//   warp 1      MMA issuer (one elected lane): S_t = Q_t K_j^T into TMEM (SS MMA), and
+//               O_t += P_t V_j with P_t read from TMEM (TS MMA).
+//   warps 2-3   TMEM allocation / release only.
+//   warps 4-7   softmax for query tile 0 (one thread per query row = TMEM lane),
+//   warps 8-11  softmax for query tile 1.
+// A work unit is a pair of adjacent query blocks (2p, 2p+1) of one (b, h); both tiles
+// share every K/V load of the merged kv-block list and ping-pong on the tensor core:
+// while one softmax group works on its S tile, the MMA warp feeds the other.
+//
+// TMEM (512 columns x 128 lanes, fp32): S0 at column 0, S1 at 128, O0 at 256, O1 at
+// 256 + D.  P_t (16-bit, two per column) overwrites the first 64 columns of S_t.
+//
+// Softmax: running max in log2 units with a lazy rescale -- O and the row sum are
+// rescaled only when the max grows by more than 8 (a factor 256), which keeps P <= 256
+// and is exact because the final division uses the same stale max.  All waits are
+// bounded; a wait that runs out sets the status word and every role unwinds.
+#include <cfloat>
+
+#include "fa_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kThreadsFwd = 384;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;         // log2 of the largest P allowed
+
+// Barrier slots.
+enum : int {
+    kBarQFull = 0,
+    kBarQEmpty = 1,
+    kBarSFull = 2,    // + tile
+    kBarPFull = 4,    // + tile
+    kBarOFull = 6,    // + tile
+    kBarOFree = 8,    // + tile
+    kBarDrain = 10,
+    kBarSlotFull = 11 // + stage, then slot-empty barriers follow
+};
+
+template <int D>
+struct Cfg {
+    static constexpr int kTileBytes = kBlock * D * 2;
+    static constexpr int kStages = (D == 64) ? 8 : 4;
+    static constexpr int kChunks = D / 64;               // 128-byte-wide TMA boxes per row
+    static constexpr int kBarSlotEmpty = kBarSlotFull + kStages;
+    static constexpr int kNumBars = kBarSlotEmpty + kStages;
+    static constexpr int kBarOff = (2 + kStages) * kTileBytes;
+    static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + alignment slack
+    // TMEM columns of S_t (P_t aliases its first 64) and O_t.
+    __device__ static constexpr uint32_t colS(int t) { return (uint32_t)t * 128u; }
+    __device__ static constexpr uint32_t colO(int t) { return 256u + (uint32_t)t * (uint32_t)D; }
+};
+
+struct Unit {
+    int b, h, pair, E;
+    const int32_t* entries;
+};
+
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
+    const int BH = p.B * p.H;
+    const int r = u / BH, bh = u - r * BH;
+    const int b = bh / p.H, h = bh - b * p.H;
+    const int mb = (p.maskB == 1) ? 0 : b, mh = (p.maskH == 1) ? 0 : h;
+    const size_t sidx = (size_t)mb * p.maskH + mh;
+    Unit un;
+    un.b = b;
+    un.h = h;
+    un.pair = __ldg(p.sched_order + sidx * p.NP + r);
+    un.E = __ldg(p.sched_count + sidx * p.NP + un.pair);
+    un.entries = p.sched_entries + (sidx * p.NP + un.pair) * (size_t)p.KVB;
+    return un;
+}
+
+// Warp-collective reader of a unit's entry list: lane l caches entry base + l.
+// Indices passed to get() must not decrease.
+struct EntryReader {
+    const int32_t* ptr;
+    int E, base, val;
+    __device__ __forceinline__ void init(const int32_t* p, int n) {
+        ptr = p;
+        E = n;
+        base = -64;
+        val = 0;
+    }
+    __device__ __forceinline__ int get(int e) {
+        const int nb = e & ~31;
+        if (nb != base) {
+            base = nb;
+            const int idx = nb + (int)(threadIdx.x & 31);
+            val = idx < E ? __ldg(ptr + idx) : 0;
+        }
+        return __shfl_sync(kFullMask, val, e & 31);
+    }
+};
+
+__device__ __forceinline__ void count_live(const int32_t* entries, int E, int& n0, int& n1) {
+    int c0 = 0, c1 = 0;
+    for (int e = threadIdx.x & 31; e < E; e += 32) {
+        const int c = __ldg(entries + e);
+        c0 += (c & kLive0) ? 1 : 0;
+        c1 += (c & kLive1) ? 1 : 0;
+    }
+    n0 = __reduce_add_sync(kFullMask, c0);
+    n1 = __reduce_add_sync(kFullMask, c1);
+}
+
+// Wait without regard to the abort flag (used to drain in-flight copies on the way out).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) break;
+    }
+    __syncwarp();
+}
+
+// ------------------------------------------------------------------ producer (warp 0)
+
+template <int D>
+__device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const CUtensorMap* tmk,
+                              const CUtensorMap* tmv, uint32_t sbase, uint32_t bars,
+                              volatile int* abort_flag) {
+    using C = Cfg<D>;
+    const int lane = threadIdx.x & 31;
+    const uint32_t sQ = sbase, sKV = sbase + 2 * C::kTileBytes;
+    auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+    auto wait = [&](int i, uint32_t par) {
+        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
+    };
+    if (lane == 0) {
+        tma_prefetch_desc(tmq);
+        tma_prefetch_desc(tmk);
+        tma_prefetch_desc(tmv);
+    }
+    uint32_t kv_pos = 0, q_iter = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(p, u);
+        if (un.E == 0) continue;
+        if (!wait(kBarQEmpty, (q_iter & 1u) ^ 1u)) { ok = false; break; }
+        const int q0 = 2 * un.pair;
+        const int nq = (q0 + 1 < p.QB) ? 2 : 1;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar(kBarQFull), (uint32_t)(nq * C::kTileBytes));
+            for (int t = 0; t < nq; ++t)
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_4d(sQ + t * C::kTileBytes + c * 16384, tmq, bar(kBarQFull), c * 64,
+                                (q0 + t) * kBlock, un.h, un.b);
+        }
+        __syncwarp();
+        ++q_iter;
+        EntryReader er;
+        er.init(un.entries, un.E);
+        for (int e = 0; e < un.E && ok; ++e) {
+            const int j = er.get(e) & 0xFFFF;
+            for (int which = 0; which < 2; ++which) {
+                const int s = (int)(kv_pos % C::kStages);
+                const uint32_t ph = (kv_pos / C::kStages) & 1u;
+                if (!wait(C::kBarSlotEmpty + s, ph ^ 1u)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(kBarSlotFull + s), (uint32_t)C::kTileBytes);
+                    const CUtensorMap* tm = which ? tmv : tmk;
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_4d(sKV + s * C::kTileBytes + c * 16384, tm, bar(kBarSlotFull + s),
+                                    c * 64, j * kBlock, un.h, un.b);
+                }
+                __syncwarp();
+                ++kv_pos;
+            }
+        }
+    }
+    if (!ok) {
+        // Let every copy already issued land before the CTA can exit.
+        const uint32_t n = kv_pos < (uint32_t)C::kStages ? kv_pos : (uint32_t)C::kStages;
+        for (uint32_t k = 0; k < n; ++k) {
+            const uint32_t pos = kv_pos - 1 - k;
+            drain_wait(bar(kBarSlotFull + (int)(pos % C::kStages)), (pos / C::kStages) & 1u);
+        }
+        if (q_iter > 0) drain_wait(bar(kBarQFull), (q_iter - 1) & 1u);
+    }
+}
+
+// ------------------------------------------------------------------ MMA issuer (warp 1)
+
+template <int D, bool BF16>
+__device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                         volatile int* abort_flag) {
+    using C = Cfg<D>;
+    const int lane = threadIdx.x & 31;
+    const uint32_t sQ = sbase, sKV = sbase + 2 * C::kTileBytes;
+    constexpr uint32_t kIdescQK = make_idesc_f16(BF16, 128, 128, false);
+    constexpr uint32_t kIdescPV = make_idesc_f16(BF16, 128, D, true);
+    auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+    auto wait = [&](int i, uint32_t par) {
+        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
+    };
+    // S_t = Q_t K^T: M = 128 query rows, N = 128 keys, K = D in steps of 16.  Both
+    // operands are K-major with 128-byte swizzle: 8-row atoms 1024 bytes apart (SBO),
+    // a step of 16 elements is 32 bytes inside the atom, and columns 64.. live in the
+    // next 16 KB box.
+    auto issue_qk = [&](int t, int slot) {
+        const uint32_t d = tmem + C::colS(t);
+        const uint32_t qa = sQ + t * C::kTileBytes, ka = sKV + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32);
+            mma_ss(d, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
+                   kIdescQK, kk > 0 ? 1u : 0u);
+        }
+    };
+    // O_t += P_t V: M = 128, N = D, K = 128 keys in steps of 16.  P_t comes from TMEM
+    // (8 columns of packed pairs per step).  V is MN-major (D contiguous): 16 keys are
+    // two 8-row atoms (SBO = 1024 bytes), 64-column boxes 16 KB apart (LBO).
+    auto issue_pv = [&](int t, int slot, bool accumulate) {
+        const uint32_t d = tmem + C::colO(t);
+        const uint32_t pa = tmem + C::colS(t);
+        const uint32_t va = sKV + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBlock / 16; ++kk) {
+            mma_ts(d, pa + (uint32_t)(kk * 8), make_sdesc_sw128(va + kk * 2048, 16384, 1024),
+                   kIdescPV, (kk > 0 || accumulate) ? 1u : 0u);
+        }
+    };
+
+    uint32_t kv_pos = 0, q_iter = 0;
+    uint32_t pf_cnt[2] = {0u, 0u}, of_cnt[2] = {0u, 0u};
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(p, u);
+        if (un.E == 0) continue;
+        int nl[2];
+        count_live(un.entries, un.E, nl[0], nl[1]);
+        if (!wait(kBarQFull, q_iter & 1u)) { ok = false; break; }
+        ++q_iter;
+        tc_fence_after();
+        const uint32_t kbase = kv_pos;
+        kv_pos += 2u * (uint32_t)un.E;
+        int ndone[2] = {0, 0};
+        EntryReader er;
+        er.init(un.entries, un.E);
+        int code = er.get(0);
+        {   // S for entry 0
+            const uint32_t pos = kbase;
+            const int s = (int)(pos % C::kStages);
+            if (!wait(kBarSlotFull + s, (pos / C::kStages) & 1u)) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) {
+                for (int t = 0; t < 2; ++t)
+                    if (code & (t ? kLive1 : kLive0)) {
+                        issue_qk(t, s);
+                        tc_commit(bar(kBarSFull + t));
+                    }
+                tc_commit(bar(C::kBarSlotEmpty + s));
+                if (un.E == 1) tc_commit(bar(kBarQEmpty));
+            }
+            __syncwarp();
+        }
+        for (int e = 0; e < un.E; ++e) {
+            const bool has_next = e + 1 < un.E;
+            const int next = has_next ? er.get(e + 1) : 0;
+            const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u, kpos = vpos + 1u;
+            const int vs = (int)(vpos % C::kStages), ks = (int)(kpos % C::kStages);
+            if (!wait(kBarSlotFull + vs, (vpos / C::kStages) & 1u)) { ok = false; break; }
+            if (has_next && !wait(kBarSlotFull + ks, (kpos / C::kStages) & 1u)) { ok = false; break; }
+            tc_fence_after();
+            for (int t = 0; t < 2; ++t) {
+                if (code & (t ? kLive1 : kLive0)) {
+                    if (!wait(kBarPFull + t, pf_cnt[t] & 1u)) { ok = false; break; }
+                    ++pf_cnt[t];
+                    if (ndone[t] == 0 && !wait(kBarOFree + t, (of_cnt[t] & 1u) ^ 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        issue_pv(t, vs, ndone[t] > 0);
+                        if (ndone[t] + 1 == nl[t]) tc_commit(bar(kBarOFull + t));
+                    }
+                    ++ndone[t];
+                }
+                if (next & (t ? kLive1 : kLive0)) {
+                    if (lane == 0) {
+                        issue_qk(t, ks);
+                        tc_commit(bar(kBarSFull + t));
+                    }
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (lane == 0) {
+                tc_commit(bar(C::kBarSlotEmpty + vs));
+                if (has_next) {
+                    tc_commit(bar(C::kBarSlotEmpty + ks));
+                    if (e + 2 == un.E) tc_commit(bar(kBarQEmpty));
+                }
+            }
+            __syncwarp();
+            code = next;
+        }
+        if (!ok) break;
+        for (int t = 0; t < 2; ++t)
+            if (nl[t] > 0) ++of_cnt[t];
+    }
+    if (!ok) {
+        // Wait for every MMA already issued before the CTA can release TMEM.
+        if (lane == 0) tc_commit(bar(kBarDrain));
+        __syncwarp();
+        drain_wait(bar(kBarDrain), 0u);
+    }
+}
+
+// ------------------------------------------------------------------ softmax (warps 4-11)
+
+template <int D, bool BF16>
+__device__ __forceinline__ void store_row_zero(const FwdParams& p, const Unit& un, int q) {
+    uint16_t* o = reinterpret_cast<uint16_t*>(p.out) + un.b * p.out_stride[0] +
+                  un.h * p.out_stride[1] + (int64_t)q * p.out_stride[2];
+#pragma unroll
+    for (int d = 0; d < D; d += 8) *reinterpret_cast<uint4*>(o + d) = make_uint4(0, 0, 0, 0);
+    if (p.lse) p.lse[((int64_t)un.b * p.H + un.h) * p.Q_LEN + q] = -INFINITY;
+}
+
+template <int D, bool BF16, bool SCORE>
+__device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t tmem,
+                             volatile int* abort_flag) {
+    using C = Cfg<D>;
+    const int wq = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant this warp may access
+    const int lane = threadIdx.x & 31;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_bits + C::colS(t);
+    const uint32_t tO = tmem + lane_bits + C::colO(t);
+    const int live_bit = t ? kLive1 : kLive0;
+    const int full_bit = t ? kFull1 : kFull0;
+    auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+    auto wait = [&](int i, uint32_t par) {
+        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
+    };
+    const bool has_softcap = SCORE && (p.score_kind & FA_SCORE_SOFTCAP);
+    const bool has_alibi = SCORE && (p.score_kind & FA_SCORE_ALIBI);
+
+    uint32_t sf_cnt = 0, of_cnt = 0;
+    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        const Unit un = decode_unit(p, u);
+        const int qblk = 2 * un.pair + t;
+        if (qblk >= p.QB) continue;
+        const int q = qblk * kBlock + row;
+        int nl0 = 0, nl1 = 0;
+        if (un.E > 0) count_live(un.entries, un.E, nl0, nl1);
+        const int nl = t ? nl1 : nl0;
+        if (nl == 0) {
+            store_row_zero<D, BF16>(p, un, q);
+            continue;
+        }
+        float slope_log2 = 0.f;
+        if (has_alibi) {
+            float slope;
+            if (p.alibi_slopes) {
+                slope = __ldg(p.alibi_slopes + un.h);
+            } else {
+                const int num = 8 * (un.h + 1);
+                slope = (num % p.H == 0) ? ldexpf(1.0f, -(num / p.H))
+                                         : exp2f(-(float)num / (float)p.H);
+            }
+            slope_log2 = slope * kLog2e;
+        }
+        float m = -INFINITY;  // running max, log2 units
+        float l = 0.f;        // running row sum of P
+        int done = 0;
+        EntryReader er;
+        er.init(un.entries, un.E);
+        bool ok = true;
+        for (int e = 0; e < un.E; ++e) {
+            const int code = er.get(e);
+            if (!(code & live_bit)) continue;
+            const int j = code & 0xFFFF;
+            const bool full = (code & full_bit) != 0;
+            if (!wait(kBarSFull + t, sf_cnt & 1u)) { ok = false; break; }
+            ++sf_cnt;
+            tc_fence_after();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, sr[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) reg_fence<32>(sr[c]);
+            float x[128];
+#pragma unroll
+            for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c >> 5][c & 31]);
+            const int kv0 = j * kBlock;
+            if constexpr (SCORE) {
+                // score_mod on every position of the tile, in log2 units; masked
+                // positions are set to -inf afterwards (the mask decides liveness).
+                const float fb = (float)(kv0 - q);
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    float y = has_softcap ? p.softcap_log2 * tanh_approx(x[c] * p.inv_softcap_scale)
+                                          : x[c] * p.scale_log2;
+                    if (has_alibi) y = fmaf(slope_log2, fb + (float)c, y);
+                    x[c] = y;
+                }
+            }
+            if (!full) {
+                int lo = 0, hi = kBlock - 1;
+                if (p.mask_kind & (FA_MASK_CAUSAL | FA_MASK_SLIDING_WINDOW)) hi = min(hi, q - kv0);
+                if (p.mask_kind & FA_MASK_SLIDING_WINDOW) lo = max(lo, q - p.window + 1 - kv0);
+                if (p.mask_kind & FA_MASK_DOCUMENT) {
+                    const int dq = __ldg(p.doc_id + q);
+                    const int4* dk = reinterpret_cast<const int4*>(p.doc_id + kv0);
+#pragma unroll
+                    for (int c4 = 0; c4 < 32; ++c4) {
+                        const int4 d4 = __ldg(dk + c4);
+                        const int c = 4 * c4;
+                        if (!(c + 0 >= lo && c + 0 <= hi && d4.x == dq)) x[c + 0] = -INFINITY;
+                        if (!(c + 1 >= lo && c + 1 <= hi && d4.y == dq)) x[c + 1] = -INFINITY;
+                        if (!(c + 2 >= lo && c + 2 <= hi && d4.z == dq)) x[c + 2] = -INFINITY;
+                        if (!(c + 3 >= lo && c + 3 <= hi && d4.w == dq)) x[c + 3] = -INFINITY;
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (c < lo || c > hi) x[c] = -INFINITY;
+                }
+            }
+            float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+            for (int c = 4; c < 128; c += 4) {
+                mx0 = fmaxf(mx0, x[c]);
+                mx1 = fmaxf(mx1, x[c + 1]);
+                mx2 = fmaxf(mx2, x[c + 2]);
+                mx3 = fmaxf(mx3, x[c + 3]);
+            }
+            float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            if constexpr (!SCORE) mt *= p.scale_log2;
+            const float m_new = fmaxf(m, mt);
+            const bool need = m_new > m + kRescaleThreshold;
+            if (__any_sync(kFullMask, need)) {
+                const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
+                if (done > 0) {
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld_32x32b_x32(tO + c * 32, o);
+                        tmem_ld_wait();
+                        reg_fence<32>(o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st_32x32b_x32(tO + c * 32, o);
+                    }
+                    tmem_st_wait();
+                }
+                if (need) {
+                    l *= alpha;
+                    m = m_new;
+                }
+            }
+            const float base = (m == -INFINITY) ? 0.f : m;
+            float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int c = half * 64 + 2 * i;
+                    float p0, p1;
+                    if constexpr (SCORE) {
+                        p0 = ex2_approx(x[c] - base);
+                        p1 = ex2_approx(x[c + 1] - base);
+                    } else {
+                        p0 = ex2_approx(fmaf(x[c], p.scale_log2, -base));
+                        p1 = ex2_approx(fmaf(x[c + 1], p.scale_log2, -base));
+                    }
+                    rs0 += p0;
+                    rs1 += p1;
+                    pk[i] = pack2<BF16>(p0, p1);
+                }
+                tmem_st_32x32b_x32(tS + half * 32, pk);
+            }
+            l += rs0 + rs1;
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar(kBarPFull + t));
+            ++done;
+        }
+        if (!ok) return;
+        // Epilogue: O / l in the output dtype, and the natural-log lse.
+        if (!wait(kBarOFull + t, of_cnt & 1u)) return;
+        ++of_cnt;
+        tc_fence_after();
+        const float inv = (l > 0.f) ? 1.0f / l : 0.f;
+        uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + un.b * p.out_stride[0] +
+                         un.h * p.out_stride[1] + (int64_t)q * p.out_stride[2];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(tO + c * 32, o);
+            tmem_ld_wait();
+            reg_fence<32>(o);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+        if (p.lse)
+            p.lse[((int64_t)un.b * p.H + un.h) * p.Q_LEN + q] =
+                (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+        tc_fence_before();
+        mbar_arrive(bar(kBarOFree + t));
+    }
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int D, bool BF16, bool SCORE>
+__global__ void __launch_bounds__(kThreadsFwd, 1)
+attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tmq,
+                const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bars = sbase + C::kBarOff;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bars + 8u * kBarQFull, 1);
+        mbar_init(bars + 8u * kBarQEmpty, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bars + 8u * (kBarSFull + t), 1);
+            mbar_init(bars + 8u * (kBarPFull + t), 128);
+            mbar_init(bars + 8u * (kBarOFull + t), 1);
+            mbar_init(bars + 8u * (kBarOFree + t), 128);
+        }
+        mbar_init(bars + 8u * kBarDrain, 1);
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(bars + 8u * (kBarSlotFull + s), 1);
+            mbar_init(bars + 8u * (C::kBarSlotEmpty + s), 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        producer_role<D>(p, &tmq, &tmk, &tmv, sbase, bars, abort_flag);
+    } else if (warp == 1) {
+        mma_role<D, BF16>(p, sbase, bars, tmem, abort_flag);
+    } else if (warp >= 4) {
+        softmax_role<D, BF16, SCORE>(p, (warp - 4) >> 2, bars, tmem, abort_flag);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+template <int D, bool BF16, bool SCORE>
+cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                     const CUtensorMap& tv, int grid, cudaStream_t stream) {
+    auto kern = attn_fwd_kernel<D, BF16, SCORE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<D>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreadsFwd, Cfg<D>::kSmemBytes, stream>>>(p, tq, tk, tv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, bool has_score,
+                            const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            int grid, cudaStream_t stream) {
+#define FA_CASE(DD, BB, SS)                                                 \
+    if (D == DD && bf16 == BB && has_score == SS)                           \
+        return launch_t<DD, BB, SS>(p, tq, tk, tv, grid, stream);
+    FA_CASE(64, true, false)
+    FA_CASE(64, true, true)
+    FA_CASE(64, false, false)
+    FA_CASE(64, false, true)
+    FA_CASE(128, true, false)
+    FA_CASE(128, true, true)
+    FA_CASE(128, false, false)
+    FA_CASE(128, false, true)
+#undef FA_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace fa

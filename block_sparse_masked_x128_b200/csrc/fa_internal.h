@@ -1,0 +1,89 @@
+// fa_internal.h -- structures shared by the host API (api.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa_b200.h"
+
+namespace fa {
+
+constexpr int kBlock = 128;          // BLOCK_SIZE: query rows and keys per tile
+constexpr int kMaxBlocks = 16384;    // q_blocks and kv_blocks limit (2M positions)
+
+// Tile classes written by the mask builder.
+constexpr int kDead = 0, kPartial = 1, kFull = 2, kAmbiguous = 3;
+
+// Schedule entry: bits 0-15 kv block, then per-tile live / full flags for the two
+// query tiles of a work unit (query blocks 2p and 2p+1).
+constexpr int kLive0 = 1 << 16, kFull0 = 1 << 17, kLive1 = 1 << 18, kFull1 = 1 << 19;
+
+// Inputs of the mask-builder kernels.
+struct MaskSpec {
+    uint32_t kind;
+    int32_t window;
+    int32_t Q_LEN, KV_LEN, QB, KVB;
+    const int32_t* doc;        // [KV_LEN] or null
+    const int32_t* doc_stats;  // [max(QB,KVB)][3] = {min, max, uniform} per block, or null
+};
+
+// Kernel parameters of the fused forward (passed by value, __grid_constant__).
+struct FwdParams {
+    int32_t B, H, Q_LEN, KV_LEN;
+    int32_t QB, KVB, NP;          // query blocks, kv blocks, work-unit pairs per (b, h)
+    int32_t maskB, maskH;         // stored mask extents (1 = broadcast)
+    int32_t n_units;              // NP * B * H
+    uint32_t mask_kind;
+    int32_t window;
+    uint32_t score_kind;
+    const int32_t* doc_id;
+    const int32_t* sched_order;   // [maskB*maskH][NP]  pairs by descending cost
+    const int32_t* sched_count;   // [maskB*maskH][NP]  entries per pair
+    const int32_t* sched_entries; // [maskB*maskH][NP][KVB]
+    float scale;                  // multiplies q k^T
+    float scale_log2;             // scale * log2(e)
+    float softcap;
+    float softcap_log2;           // softcap * log2(e)
+    float inv_softcap_scale;      // scale / softcap
+    const float* alibi_slopes;    // device [H] or null (then 2^(-8(h+1)/H))
+    void* out;
+    int64_t out_stride[3];        // B, H, S strides in elements (D stride is 1)
+    float* lse;                   // [B][H][Q_LEN] or null
+    int32_t* status;              // device status word (1 = a bounded wait ran out)
+};
+
+cudaError_t launch_mask_build(const MaskSpec& spec, int separate_full, int maskBH, int NP,
+                              int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
+                              int32_t* full_idx, int32_t* doc_stats, int32_t* sched_count,
+                              int32_t* sched_cost, int32_t* sched_entries, int32_t* sched_order,
+                              cudaStream_t stream);
+
+cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, bool has_score,
+                            const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            int grid, cudaStream_t stream);
+
+}  // namespace fa
+
+struct fa_block_mask {
+    uint32_t mask_kind;
+    int32_t window;
+    int32_t separate_full;
+    int32_t B, H;            // stored extents (1 when broadcast)
+    int32_t Q_LEN, KV_LEN, QB, KVB, NP;
+    int device;
+    void* dev_base;
+    int32_t* kv_num;
+    int32_t* kv_idx;
+    int32_t* full_num;
+    int32_t* full_idx;
+    int32_t* doc;
+    int32_t* doc_stats;
+    int32_t* sched_count;
+    int32_t* sched_cost;
+    int32_t* sched_entries;
+    int32_t* sched_order;
+    int32_t* status;
+};

@@ -1,0 +1,287 @@
+// mask_builder.cu -- block-mask construction on the GPU.
+//
+// Follows "tensorplay.nn.attention.create_block_mask" (Parameters: BLOCK_SIZE,
+// separate_full_blocks) and "How to Use FlexAttention on Apple Silicon" ("The two hooks":
+// fully masked blocks are skipped; "Mask 1": build once, broadcast over B and H).
+//
+// Three steps, all integer work:
+//   1. classify_compact_kernel: one CTA per (stored b/h, query block).  Each thread
+//      classifies one kv block at a time as dead / partial / full.  The causal and
+//      sliding-window predicates depend only on d = q - kv, which takes every integer
+//      value between its extremes over a rectangular tile, so interval arithmetic on d
+//      classifies those tiles exactly.  The document predicate is resolved from
+//      per-block (min, max, uniform) statistics where they decide it; the remaining
+//      tiles are evaluated element by element by the whole CTA.  Live tiles are then
+//      compacted into ascending lists with warp ballots and popc prefix sums.
+//   2. schedule_kernel: one CTA per work unit (a pair of adjacent query blocks) merges
+//      the two tiles' partial and full lists into one ascending list of kv blocks with
+//      per-tile live/full flags, so the forward kernel loads each K/V tile once for both
+//      query tiles.  The unit's cost is the number of live tiles it holds.
+//   3. lpt_order_kernel: ranks the units of each stored (b, h) by descending cost (ties
+//      by index) so the persistent forward kernel hands the longest units out first.
+#include <climits>
+
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+constexpr int kThreads = 128;  // == kBlock: one thread per query row when resolving a tile
+
+__global__ void __launch_bounds__(kThreads) doc_block_stats_kernel(const int32_t* __restrict__ doc,
+                                                                  int len, int nblk,
+                                                                  int32_t* __restrict__ stats) {
+    const int blk = blockIdx.x;
+    if (blk >= nblk) return;
+    const int s0 = blk * kBlock;
+    const int n = min(kBlock, len - s0);
+    int mn = INT_MAX, mx = INT_MIN;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int d = doc[s0 + i];
+        mn = min(mn, d);
+        mx = max(mx, d);
+    }
+    mn = __reduce_min_sync(0xffffffffu, mn);
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    __shared__ int smn[kThreads / 32], smx[kThreads / 32];
+    if ((threadIdx.x & 31) == 0) {
+        smn[threadIdx.x >> 5] = mn;
+        smx[threadIdx.x >> 5] = mx;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kThreads / 32; ++w) {
+            mn = min(mn, smn[w]);
+            mx = max(mx, smx[w]);
+        }
+        stats[3 * blk + 0] = mn;
+        stats[3 * blk + 1] = mx;
+        stats[3 * blk + 2] = (mn == mx) ? 1 : 0;
+    }
+}
+
+// Allowed range of d = q - kv from the interval predicates (causal, sliding window).
+__device__ __forceinline__ void interval_bounds(const MaskSpec& m, long long& lo, long long& hi) {
+    lo = LLONG_MIN / 4;
+    hi = LLONG_MAX / 4;
+    if (m.kind & FA_MASK_CAUSAL) lo = lo > 0 ? lo : 0;
+    if (m.kind & FA_MASK_SLIDING_WINDOW) {
+        lo = lo > 0 ? lo : 0;
+        hi = hi < (long long)m.window - 1 ? hi : (long long)m.window - 1;
+    }
+}
+
+__device__ int classify_fast(const MaskSpec& m, int i, int j) {
+    const int qs = i * kBlock, qe = min(qs + kBlock, m.Q_LEN) - 1;
+    const int ks = j * kBlock, ke = min(ks + kBlock, m.KV_LEN) - 1;
+    const bool ragged = (qe - qs + 1 < kBlock) || (ke - ks + 1 < kBlock);
+    long long lo, hi;
+    interval_bounds(m, lo, hi);
+    const long long dmin = (long long)qs - ke, dmax = (long long)qe - ks;
+    if (dmax < lo || dmin > hi) return kDead;
+    const bool interval_full = dmin >= lo && dmax <= hi;
+    if (!(m.kind & FA_MASK_DOCUMENT)) return (interval_full && !ragged) ? kFull : kPartial;
+    const int32_t* qst = m.doc_stats + 3 * i;
+    const int32_t* kst = m.doc_stats + 3 * j;
+    if (qst[1] < kst[0] || kst[1] < qst[0]) return kDead;   // id ranges disjoint
+    if (qst[2] && kst[2]) {                                  // both blocks hold one id
+        if (qst[0] != kst[0]) return kDead;
+        return (interval_full && !ragged) ? kFull : kPartial;
+    }
+    return kAmbiguous;
+}
+
+// Element-by-element classification of one tile by the whole CTA (thread r = query row r).
+__device__ int resolve_tile(const MaskSpec& m, int i, int j) {
+    long long lo, hi;
+    interval_bounds(m, lo, hi);
+    const int q = i * kBlock + threadIdx.x;
+    const bool q_in = q < m.Q_LEN;
+    const int dq = (q_in && m.doc) ? m.doc[q] : 0;
+    bool any = false, all = true;
+    for (int c = 0; c < kBlock; ++c) {
+        const int kv = j * kBlock + c;
+        bool live = q_in && kv < m.KV_LEN;
+        if (live) {
+            const long long d = (long long)q - kv;
+            live = d >= lo && d <= hi;
+            if (live && (m.kind & FA_MASK_DOCUMENT)) live = (m.doc[kv] == dq);
+        }
+        any |= live;
+        all &= live;
+    }
+    const int a = __syncthreads_or(any ? 1 : 0);
+    const int f = __syncthreads_and(all ? 1 : 0);
+    return !a ? kDead : (f ? kFull : kPartial);
+}
+
+__global__ void __launch_bounds__(kThreads)
+classify_compact_kernel(MaskSpec m, int separate_full, int32_t* __restrict__ kv_num,
+                        int32_t* __restrict__ kv_idx, int32_t* __restrict__ full_num,
+                        int32_t* __restrict__ full_idx) {
+    const int i = blockIdx.x;
+    const int bh = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int s_cls[kThreads];
+    __shared__ int s_amb[kThreads];
+    __shared__ int s_namb;
+    __shared__ int s_wp[kThreads / 32], s_wf[kThreads / 32];
+
+    const size_t row = (size_t)bh * m.QB + i;
+    int32_t* my_kv = kv_idx + row * m.KVB;
+    int32_t* my_full = full_idx + row * m.KVB;
+    int np = 0, nf = 0;
+    for (int jb = 0; jb < m.KVB; jb += kThreads) {
+        const int j = jb + tid;
+        int cls = (j < m.KVB) ? classify_fast(m, i, j) : kDead;
+        if (tid == 0) s_namb = 0;
+        __syncthreads();
+        if (cls == kAmbiguous) s_amb[atomicAdd(&s_namb, 1)] = tid;
+        s_cls[tid] = cls;
+        __syncthreads();
+        const int namb = s_namb;
+        for (int a = 0; a < namb; ++a) {
+            const int t = s_amb[a];
+            const int c = resolve_tile(m, i, jb + t);
+            if (tid == 0) s_cls[t] = c;
+        }
+        __syncthreads();
+        cls = s_cls[tid];
+        if (!separate_full && cls == kFull) cls = kPartial;
+        const unsigned bp = __ballot_sync(0xffffffffu, cls == kPartial);
+        const unsigned bf = __ballot_sync(0xffffffffu, cls == kFull);
+        if (lane == 0) {
+            s_wp[warp] = __popc(bp);
+            s_wf[warp] = __popc(bf);
+        }
+        __syncthreads();
+        int op = np, of = nf, tp = 0, tf = 0;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            if (w < warp) {
+                op += s_wp[w];
+                of += s_wf[w];
+            }
+            tp += s_wp[w];
+            tf += s_wf[w];
+        }
+        const unsigned lt = (1u << lane) - 1u;
+        if (cls == kPartial) my_kv[op + __popc(bp & lt)] = j;
+        if (cls == kFull) my_full[of + __popc(bf & lt)] = j;
+        np += tp;
+        nf += tf;
+        __syncthreads();
+    }
+    for (int t = np + tid; t < m.KVB; t += kThreads) my_kv[t] = 0;
+    for (int t = nf + tid; t < m.KVB; t += kThreads) my_full[t] = 0;
+    if (tid == 0) {
+        kv_num[row] = np;
+        full_num[row] = nf;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+schedule_kernel(int QB, int KVB, int NP, const int32_t* __restrict__ kv_num,
+                const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ full_num,
+                const int32_t* __restrict__ full_idx, int32_t* __restrict__ sched_count,
+                int32_t* __restrict__ sched_cost, int32_t* __restrict__ sched_entries) {
+    extern __shared__ uint8_t s_code[];  // one byte of flags per kv block
+    const int p = blockIdx.x, bh = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int s_w[kThreads / 32], s_l0[kThreads / 32], s_l1[kThreads / 32];
+    for (int j = tid; j < KVB; j += kThreads) s_code[j] = 0;
+    __syncthreads();
+    for (int t = 0; t < 2; ++t) {
+        const int i = 2 * p + t;
+        if (i >= QB) break;
+        const size_t row = (size_t)bh * QB + i;
+        const uint8_t live = (uint8_t)(t ? (kLive1 >> 16) : (kLive0 >> 16));
+        const uint8_t full = (uint8_t)(t ? (kFull1 >> 16) : (kFull0 >> 16));
+        const int n_p = kv_num[row], n_f = full_num[row];
+        for (int n = tid; n < n_p; n += kThreads) {
+            const int j = kv_idx[row * KVB + n];
+            if (j >= 0 && j < KVB) s_code[j] |= live;
+        }
+        __syncthreads();
+        for (int n = tid; n < n_f; n += kThreads) {
+            const int j = full_idx[row * KVB + n];
+            if (j >= 0 && j < KVB) s_code[j] |= (uint8_t)(live | full);
+        }
+        __syncthreads();
+    }
+    const size_t unit = (size_t)bh * NP + p;
+    int32_t* out = sched_entries + unit * KVB;
+    int cnt = 0, l0 = 0, l1 = 0;
+    for (int jb = 0; jb < KVB; jb += kThreads) {
+        const int j = jb + tid;
+        const int c = (j < KVB) ? s_code[j] : 0;
+        const unsigned b = __ballot_sync(0xffffffffu, c != 0);
+        const unsigned b0 = __ballot_sync(0xffffffffu, (c & (kLive0 >> 16)) != 0);
+        const unsigned b1 = __ballot_sync(0xffffffffu, (c & (kLive1 >> 16)) != 0);
+        if (lane == 0) {
+            s_w[warp] = __popc(b);
+            s_l0[warp] = __popc(b0);
+            s_l1[warp] = __popc(b1);
+        }
+        __syncthreads();
+        int off = cnt, tot = 0;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            if (w < warp) off += s_w[w];
+            tot += s_w[w];
+            l0 += s_l0[w];
+            l1 += s_l1[w];
+        }
+        if (c != 0) out[off + __popc(b & ((1u << lane) - 1u))] = j | (c << 16);
+        cnt += tot;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        sched_count[unit] = cnt;
+        sched_cost[unit] = l0 + l1;
+    }
+}
+
+__global__ void __launch_bounds__(1024) lpt_order_kernel(int NP, const int32_t* __restrict__ cost,
+                                                        int32_t* __restrict__ order) {
+    extern __shared__ int s_cost[];
+    const int bh = blockIdx.x;
+    for (int p = threadIdx.x; p < NP; p += blockDim.x) s_cost[p] = cost[(size_t)bh * NP + p];
+    __syncthreads();
+    for (int p = threadIdx.x; p < NP; p += blockDim.x) {
+        const int c = s_cost[p];
+        int rank = 0;
+        for (int o = 0; o < NP; ++o) {
+            const int co = s_cost[o];
+            rank += (co > c) || (co == c && o < p);
+        }
+        order[(size_t)bh * NP + rank] = p;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_mask_build(const MaskSpec& spec, int separate_full, int maskBH, int NP,
+                              int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
+                              int32_t* full_idx, int32_t* doc_stats, int32_t* sched_count,
+                              int32_t* sched_cost, int32_t* sched_entries, int32_t* sched_order,
+                              cudaStream_t stream) {
+    if (spec.kind & FA_MASK_DOCUMENT) {
+        const int nblk = spec.QB > spec.KVB ? spec.QB : spec.KVB;
+        doc_block_stats_kernel<<<nblk, kThreads, 0, stream>>>(spec.doc, spec.KV_LEN, nblk,
+                                                              doc_stats);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    classify_compact_kernel<<<dim3(spec.QB, maskBH), kThreads, 0, stream>>>(
+        spec, separate_full, kv_num, kv_idx, full_num, full_idx);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    schedule_kernel<<<dim3(NP, maskBH), kThreads, spec.KVB, stream>>>(
+        spec.QB, spec.KVB, NP, kv_num, kv_idx, full_num, full_idx, sched_count, sched_cost,
+        sched_entries);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    lpt_order_kernel<<<maskBH, 1024, NP * (int)sizeof(int), stream>>>(NP, sched_cost, sched_order);
+    return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,181 @@
+/*
+ * fa_b200.h -- C ABI of the B200 (sm_100a) block-sparse masked attention library.
+ *
+ * Two operations make up the path:
+ *
+ *   fa_create_block_mask   evaluates a fixed mask_mod over the 128 x 128 tile grid
+ *                          and emits, per query block, the ascending lists of
+ *                          partially masked and fully unmasked key/value blocks
+ *                          ("tensorplay.nn.attention.create_block_mask", Parameters:
+ *                          BLOCK_SIZE, separate_full_blocks; "How to Use FlexAttention
+ *                          on Apple Silicon", sections "The two hooks" and "Mask 1").
+ *   fa_forward             one fused attention forward over the live tiles only:
+ *                          mask_mod on partial tiles, score_mod on live scores, online
+ *                          softmax, O and the log-sum-exp written out; the N x N score
+ *                          matrix never exists ("How to Use FlexAttention on Apple
+ *                          Silicon", "The two hooks" and "Bonus: a score_mod for
+ *                          soft-capping").
+ *
+ * Conventions shared by every call:
+ *   - All tensor data pointers are DEVICE pointers owned by the caller unless stated.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Calls are asynchronous on that stream; they never synchronise it except
+ *     fa_get_device_status.
+ *   - Every call returns a status and never throws or aborts across the ABI.  All
+ *     argument checks happen before any launch; on an error nothing is launched and
+ *     no output is written.  fa_last_error_message() gives a one-line reason.
+ *   - Library objects are not thread-safe against concurrent destroy; concurrent
+ *     fa_forward calls on one mask from different streams are allowed (the mask is
+ *     read-only for them).
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fa_status {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, bad flag bits, mismatched tensors */
+    FA_ERR_UNSUPPORTED = 2,   /* valid request outside what the kernels implement */
+    FA_ERR_CUDA = 3,          /* a CUDA runtime/driver call or a launch failed */
+    FA_ERR_OOM = 4,           /* device allocation failed */
+    FA_ERR_TIMEOUT = 5,       /* a device-side wait ran past its limit (see fa_get_device_status) */
+    FA_ERR_INTERNAL = 6
+} fa_status_t;
+
+/* mask_mod kinds: bit flags, OR-ed together meaning the conjunction (AND) of the
+ * predicates ("How to Use FlexAttention on Apple Silicon", Masks 2 and 3 combine
+ * predicates with &).  0 means every pair is allowed. */
+#define FA_MASK_CAUSAL          1u   /* q_idx >= kv_idx                        ("Mask 1: causal")          */
+#define FA_MASK_SLIDING_WINDOW  2u   /* 0 <= q_idx - kv_idx < window           ("Sliding-Window Self-Attention",
+                                        "State the boundary precisely"; includes causality)               */
+#define FA_MASK_DOCUMENT        4u   /* doc_id[q_idx] == doc_id[kv_idx]        ("Mask 3: document-packed") */
+
+/* score_mod kinds: bit flags.  With both, the soft-cap is applied first and the
+ * ALiBi bias is added to the capped score. */
+#define FA_SCORE_NONE     0u
+#define FA_SCORE_SOFTCAP  1u   /* softcap * tanh(score / softcap)  ("Bonus: a score_mod for soft-capping") */
+#define FA_SCORE_ALIBI    2u   /* score + slope_h * (kv_idx - q_idx)  (additive distance bias, "The two hooks") */
+
+#define FA_DTYPE_F16   0
+#define FA_DTYPE_BF16  1
+
+typedef struct fa_mask_params {
+    int32_t        window;                /* W > 0, used when FA_MASK_SLIDING_WINDOW is set        */
+    const int32_t* doc_id;                /* device, KV_LEN int32 ids (FA_MASK_DOCUMENT); requires
+                                             Q_LEN == KV_LEN.  Copied: the caller may free it after
+                                             fa_create_block_mask returns and the stream has run.  */
+    int32_t        separate_full_blocks;  /* 1: fully unmasked tiles go to the full_* lists so the
+                                             kernel skips mask_mod there; 0: every live tile is
+                                             listed as partial ("create_block_mask", Parameters)   */
+} fa_mask_params_t;
+
+typedef struct fa_score_params {
+    float        softcap;        /* > 0 when FA_SCORE_SOFTCAP is set (30 in the soft-capping example) */
+    const float* alibi_slopes;   /* device [H] fp32, or NULL for the slopes 2^(-8(h+1)/H)              */
+} fa_score_params_t;
+
+/* A (B, H, S, D) tensor: batch, heads, sequence, head_dim, the layout shared with
+ * scaled_dot_product_attention ("How to Use FlexAttention on Apple Silicon", Setup). */
+typedef struct fa_tensor {
+    void*   data;        /* device pointer, 16-byte aligned                         */
+    int32_t dtype;       /* FA_DTYPE_F16 or FA_DTYPE_BF16                           */
+    int64_t B, H, S, D;
+    int64_t stride[4];   /* element strides of B, H, S, D; stride[3] must be 1 and the
+                            others positive multiples of 8 (16 bytes)               */
+} fa_tensor_t;
+
+typedef struct fa_block_mask fa_block_mask_t;   /* opaque, owned by the library */
+
+/* Read-only view of a block mask (all pointers are device pointers owned by the mask). */
+typedef struct fa_block_mask_info {
+    int32_t  B, H;              /* stored extents: 1 where the mask was created broadcast */
+    int32_t  Q_LEN, KV_LEN, BLOCK_SIZE;
+    int32_t  q_blocks, kv_blocks;
+    uint32_t mask_kind;
+    int32_t  window;
+    int32_t  separate_full_blocks;
+    const int32_t* kv_num_blocks;       /* [B][H][q_blocks]            partial tiles per query block   */
+    const int32_t* kv_indices;          /* [B][H][q_blocks][kv_blocks] ascending, zero padded          */
+    const int32_t* full_kv_num_blocks;  /* [B][H][q_blocks]            full tiles per query block      */
+    const int32_t* full_kv_indices;     /* [B][H][q_blocks][kv_blocks] ascending, zero padded          */
+} fa_block_mask_info_t;
+
+/*
+ * fa_create_block_mask -- build the block mask of a fixed mask_mod on the GPU.
+ *
+ * Follows "tensorplay.nn.attention.create_block_mask" (signature and Parameters) and
+ * "How to Use FlexAttention on Apple Silicon" ("Mask 1": B=None, H=None broadcast the
+ * mask; build it once and reuse it).  A tile is dead when no pair in it is allowed,
+ * full when every pair is allowed and the tile lies wholly inside Q_LEN x KV_LEN, and
+ * partial otherwise.  Lists hold ascending kv-block indices padded with 0.
+ *
+ *   mask_kind   OR of FA_MASK_* bits (0 = no mask)
+ *   params      may be NULL when mask_kind needs neither window nor doc_id
+ *               (separate_full_blocks then defaults to 1)
+ *   B, H        batch and head extents; 0 means broadcast (stored as 1)
+ *   Q_LEN, KV_LEN > 0;  BLOCK_SIZE must be 128 (else FA_ERR_UNSUPPORTED)
+ *   out_mask    receives the new mask; release it with fa_destroy_block_mask
+ *
+ * Work is enqueued on `stream`; the mask may be used by fa_forward on the same stream
+ * at once, or on another stream after synchronising.  Errors: FA_ERR_INVALID_ARG,
+ * FA_ERR_UNSUPPORTED, FA_ERR_OOM, FA_ERR_CUDA.
+ */
+fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* params,
+                                 int32_t B, int32_t H, int32_t Q_LEN, int32_t KV_LEN,
+                                 int32_t BLOCK_SIZE, void* stream, fa_block_mask_t** out_mask);
+
+/*
+ * fa_forward -- fused block-sparse attention forward.
+ *
+ * out = softmax(mask(score_mod(scale * q k^T))) v  and  lse = log(sum(exp(...))) per query
+ * row, natural log, fp32 ("How to Use FlexAttention on Apple Silicon", "The two hooks":
+ * mask_mod decides which pairs live, score_mod changes only live scores).  Only the
+ * tiles the mask lists are visited; mask_mod is evaluated only on partial tiles.
+ *
+ *   q           (B, H, Q_LEN, D);  k, v (B, H, KV_LEN, D);  all the same dtype
+ *   block_mask  from fa_create_block_mask with matching Q_LEN/KV_LEN and with B, H
+ *               equal to q's or broadcast
+ *   score_mod_kind / params   FA_SCORE_* bits; params may be NULL for FA_SCORE_NONE
+ *   scale       multiplies q k^T before score_mod; <= 0 selects 1/sqrt(D)
+ *   out         (B, H, Q_LEN, D), q's dtype, caller-owned
+ *   lse         device fp32 [B][H][Q_LEN] contiguous, or NULL to skip it
+ *
+ * Supported now: D in {64, 128}; Q_LEN and KV_LEN multiples of 128 (else
+ * FA_ERR_UNSUPPORTED).  A query row with no allowed key gets out = 0, lse = -inf.
+ * Device-side waits are bounded; a wait that runs out sets the mask's status word
+ * (read it with fa_get_device_status) and the kernel returns early.
+ */
+fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tensor_t* v,
+                       const fa_block_mask_t* block_mask, uint32_t score_mod_kind,
+                       const fa_score_params_t* params, float scale,
+                       fa_tensor_t* out, float* lse, void* stream);
+
+/* Fill `info` with the mask's extents and device pointers.  FA_ERR_INVALID_ARG on NULL. */
+fa_status_t fa_block_mask_get(const fa_block_mask_t* block_mask, fa_block_mask_info_t* info);
+
+/*
+ * Synchronise `stream`, read and clear the device status word that kernels using this
+ * mask write when a bounded device-side wait runs out.  Returns FA_OK, FA_ERR_TIMEOUT,
+ * or FA_ERR_CUDA if the stream itself reports an error.
+ */
+fa_status_t fa_get_device_status(const fa_block_mask_t* block_mask, void* stream);
+
+/* Free a mask (NULL is ignored).  The caller must ensure no enqueued work still uses it. */
+void fa_destroy_block_mask(fa_block_mask_t* block_mask);
+
+/* Static string naming a status code. */
+const char* fa_status_string(fa_status_t status);
+
+/* One-line description of the last error returned on the calling thread ("" if none). */
+const char* fa_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

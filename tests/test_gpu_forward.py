@@ -1,0 +1,203 @@
+"""Fused forward on the GPU against the float64 oracle on the same seeded inputs.
+
+Oracle-sized cases compare every output element; full-size workloads (in the launch
+configuration the benchmark times) compare sampled query rows the oracle computes one by
+one.  Bit-exact checks cover what the method fixes exactly: a window of one returns V, keys
+outside a row's mask cannot change it, packed documents equal separate runs, and the
+separate_full_blocks setting does not change the arithmetic.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from gpu_common import compare, fa_module, gpu_block_mask, run_gpu, run_oracle, workload_inputs
+
+pytestmark = pytest.mark.gpu
+
+C, SW, DOC = wl.MASK_CAUSAL, wl.MASK_SLIDING_WINDOW, wl.MASK_DOCUMENT
+
+# Oracle-sized versions of the five workloads (several tiles and pairs, ragged doc edges).
+SMALL = [
+    wl.WORKLOADS[0],
+    wl.WORKLOADS[1].scaled(S=1024),
+    wl.WORKLOADS[2].scaled(S=2048, H=4),
+    wl.WORKLOADS[3].scaled(S=2048, H=4),
+    wl.WORKLOADS[4].scaled(S=2048),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name + f"_S{w.S}" for w in SMALL])
+def test_forward_matches_oracle_everywhere(w):
+    q, k, v = wl.make_qkv(w)
+    doc = wl.make_doc_ids(w)
+    out, lse, _ = run_gpu(w, q, k, v, doc)
+    O, L = run_oracle(w, q, k, v, doc)
+    compare(out, lse, O, L)
+
+
+def _sample_rows(S, seed, n_random=8):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, 129, 255, 256, S // 2 - 1, S // 2, S - 129, S - 128, S - 2, S - 1]
+    return sorted(set(fixed) | set(rng.integers(0, S, n_random).tolist()))
+
+
+@pytest.mark.parametrize("w", wl.WORKLOADS, ids=[w.name for w in wl.WORKLOADS])
+def test_forward_full_size_sampled_rows(w):
+    q, k, v, doc = workload_inputs(w)
+    out, lse, _ = run_gpu(w, q, k, v, doc)
+    rows = _sample_rows(w.S, w.seed)
+    if doc is not None:   # rows around every document boundary
+        starts = np.flatnonzero(np.diff(doc)) + 1
+        rows = sorted(set(rows) | {int(s) + d for s in starts for d in (-1, 0, 1)})
+    O, L = run_oracle(w, q, k, v, doc, rows=rows)
+    compare(out, lse, O, L, rows=rows)
+
+
+@pytest.mark.parametrize("D,dtype", [(64, torch.float16), (64, torch.bfloat16), (128, torch.bfloat16),
+                                     (128, torch.float16)])
+def test_window_one_returns_v_exactly(D, dtype):
+    fa = fa_module()
+    g = torch.Generator().manual_seed(11)
+    q, k, v = (torch.randn(2, 3, 512, D, generator=g).to(dtype).cuda() for _ in range(3))
+    bm = gpu_block_mask(SW, None, None, 512, 512, 1)
+    out, lse = fa.flex_attention(q, k, v, bm)
+    assert torch.equal(out, v)
+    s_ii = (q.double() * k.double()).sum(-1) / np.sqrt(D)
+    assert (lse.double() - s_ii).abs().max().item() < 1e-4
+
+
+def test_keys_outside_the_window_cannot_change_a_row():
+    # "The last query cannot read row zero through this single layer."
+    fa = fa_module()
+    w = wl.WORKLOADS[0]
+    q, k, v = (t.cuda() for t in wl.make_qkv(w))
+    bm = gpu_block_mask(w.mask_kind, None, None, 512, 512, w.window)
+    out, lse = fa.flex_attention(q, k, v, bm, scale=w.scale)
+    k2, v2 = k.clone(), v.clone()
+    k2[:, :, :256] += 3.0           # rows >= 384 see only keys 257..511
+    v2[:, :, :256] -= 5.0
+    out2, lse2 = fa.flex_attention(q, k2, v2, bm, scale=w.scale)
+    assert torch.equal(out[:, :, 384:], out2[:, :, 384:])
+    assert torch.equal(lse[:, :, 384:], lse2[:, :, 384:])
+    assert not torch.equal(out[:, :, :256], out2[:, :, :256])
+
+
+def test_packed_documents_equal_separate_runs():
+    fa = fa_module()
+    lengths = [256, 384, 128, 256]
+    doc = wl.doc_ids_from_lengths(lengths)
+    g = torch.Generator().manual_seed(5)
+    q, k, v = (torch.randn(1, 4, 1024, 128, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    bm = gpu_block_mask(C | DOC, None, None, 1024, 1024, 0, doc)
+    out, lse = fa.flex_attention(q, k, v, bm)
+    start = 0
+    for L in lengths:
+        sl = slice(start, start + L)
+        bmd = gpu_block_mask(C, None, None, L, L)
+        od, ld = fa.flex_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(),
+                                   v[:, :, sl].contiguous(), bmd)
+        assert torch.equal(out[:, :, sl], od)
+        assert torch.equal(lse[:, :, sl], ld)
+        start += L
+
+
+@pytest.mark.parametrize("kind,window", [(C, 0), (C | SW, 300), (C | DOC, 0)])
+def test_separate_full_blocks_does_not_change_the_result(kind, window):
+    fa = fa_module()
+    doc = wl.doc_ids_from_lengths([700, 900, 448]) if kind & DOC else None
+    g = torch.Generator().manual_seed(6)
+    q, k, v = (torch.randn(1, 2, 2048, 64, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    a = fa.flex_attention(q, k, v, gpu_block_mask(kind, None, None, 2048, 2048, window, doc, True))
+    b = fa.flex_attention(q, k, v, gpu_block_mask(kind, None, None, 2048, 2048, window, doc, False))
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_strided_layout_equals_contiguous():
+    fa = fa_module()
+    g = torch.Generator().manual_seed(8)
+    base = [torch.randn(2, 768, 3, 128, generator=g).to(torch.bfloat16).cuda() for _ in range(3)]
+    q, k, v = (t.transpose(1, 2) for t in base)            # (B, H, S, D) views, S stride H*D
+    bm = gpu_block_mask(C, None, None, 768, 768)
+    out_view = torch.empty(2, 768, 3, 128, dtype=torch.bfloat16, device="cuda").transpose(1, 2)
+    o1, l1 = fa.flex_attention(q, k, v, bm, out=out_view)
+    o2, l2 = fa.flex_attention(q.contiguous(), k.contiguous(), v.contiguous(), bm)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_rows_without_live_keys_give_zero_and_minus_inf():
+    w = wl.Workload("swa128_q512_kv128", B=1, H=2, S=512, D=64, dtype="bf16",
+                    mask_kind=SW, window=128, seed=21)
+    fa = fa_module()
+    g = torch.Generator().manual_seed(21)
+    q = torch.randn(1, 2, 512, 64, generator=g).to(torch.bfloat16)
+    k = torch.randn(1, 2, 128, 64, generator=g).to(torch.bfloat16)
+    v = torch.randn(1, 2, 128, 64, generator=g).to(torch.bfloat16)
+    bm = gpu_block_mask(SW, None, None, 512, 128, 128)
+    out, lse = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm)
+    O, L = run_oracle(w, q, k, v)
+    compare(out, lse, O, L)
+    assert torch.all(out[:, :, 255:] == 0) and torch.all(torch.isinf(lse[:, :, 255:]))
+
+
+@pytest.mark.parametrize("Q,KV,kind,window", [(256, 640, C, 0), (640, 256, C, 0), (384, 1024, SW, 200)])
+def test_query_and_key_lengths_may_differ(Q, KV, kind, window):
+    w = wl.Workload("qkv_lengths", B=1, H=2, S=Q, D=128, dtype="bf16", mask_kind=kind,
+                    window=window, seed=22)
+    fa = fa_module()
+    g = torch.Generator().manual_seed(22)
+    q = torch.randn(1, 2, Q, 128, generator=g).to(torch.bfloat16)
+    k = torch.randn(1, 2, KV, 128, generator=g).to(torch.bfloat16)
+    v = torch.randn(1, 2, KV, 128, generator=g).to(torch.bfloat16)
+    bm = gpu_block_mask(kind, None, None, Q, KV, window)
+    out, lse = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm)
+    O, L = run_oracle(w, q, k, v)
+    compare(out, lse, O, L)
+
+
+def test_per_head_mask_equals_broadcast_mask():
+    fa = fa_module()
+    g = torch.Generator().manual_seed(9)
+    q, k, v = (torch.randn(2, 3, 1024, 64, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    a = fa.flex_attention(q, k, v, gpu_block_mask(C | SW, None, None, 1024, 1024, 256))
+    b = fa.flex_attention(q, k, v, gpu_block_mask(C | SW, 2, 3, 1024, 1024, 256))
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("score_kind", [wl.SCORE_SOFTCAP, wl.SCORE_ALIBI, wl.SCORE_SOFTCAP | wl.SCORE_ALIBI])
+@pytest.mark.parametrize("D,dtype", [(64, "fp16"), (128, "bf16")])
+def test_score_mods(score_kind, D, dtype):
+    w = wl.Workload("score_mods", B=1, H=4, S=768, D=D, dtype=dtype, mask_kind=C,
+                    score_kind=score_kind, softcap=5.0, seed=23)
+    q, k, v = wl.make_qkv(w)
+    q = q * 3   # large enough scores for the cap to bend them
+    out, lse, _ = run_gpu(w, q, k, v)
+    O, L = run_oracle(w, q, k, v)
+    compare(out, lse, O, L)
+
+
+def test_explicit_alibi_slopes():
+    fa = fa_module()
+    w = wl.Workload("alibi_slopes", B=1, H=4, S=512, D=128, dtype="bf16", mask_kind=C,
+                    score_kind=wl.SCORE_ALIBI, seed=24)
+    q, k, v = wl.make_qkv(w)
+    slopes = np.array([0.3, 0.05, 1.0, 0.0], dtype=np.float32)
+    bm = gpu_block_mask(C, None, None, 512, 512)
+    out, lse = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm, score_mod=wl.SCORE_ALIBI,
+                                 alibi_slopes=torch.from_numpy(slopes).cuda())
+    sm = oracle.alibi(slopes.astype(np.float64))
+    O, L = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), oracle.causal, sm)
+    compare(out, lse, O, L)
+
+
+def test_lse_may_be_omitted_and_runs_are_deterministic():
+    fa = fa_module()
+    w = wl.WORKLOADS[1].scaled(S=1024, H=4)
+    q, k, v = (t.cuda() for t in wl.make_qkv(w))
+    bm = gpu_block_mask(C, None, None, 1024, 1024)
+    o1, _ = fa.flex_attention(q, k, v, bm, return_lse=False)
+    o2, l2 = fa.flex_attention(q, k, v, bm)
+    assert torch.equal(o1, o2)
+    o3, l3 = fa.flex_attention(q, k, v, bm)
+    assert torch.equal(o2, o3) and torch.equal(l2, l3)
