@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark: live-position attention forward TFLOP/s of the block-sparse kernel on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one fused forward (``fa_forward``) over one batch of the workload with the block
+mask already built: the pages build the mask once and reuse it across forward passes, so the
+mask build is timed separately (``mask_build_ms``) and is not part of the metric.  FLOPs are
+4 * D * (exact number of live mask positions) * B * H per step; masked positions inside live
+tiles and dead tiles do not count.
+
+Under torchrun (N > 1) every rank runs its own independent batch of the workload (data
+parallel, weak scaling, no collective on the data path); time is the max over ranks of the
+CUDA-event time and ``value`` counts the work of all ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as wl  # noqa: E402
+
+DEFAULT_WORKLOAD = wl.WORKLOADS[1].name    # 8k dense causal, D = 64, bf16
+METRIC = "live-position attention fwd TFLOP/s"
+UNIT = "TFLOP/s"
+L2_FLUSH_BYTES = 512 << 20                  # > 126 MB of L2
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+# ---------------------------------------------------------------- work accounting
+
+def live_positions_per_head(w: wl.Workload, doc=None) -> int:
+    """Exact count of allowed (q, kv) pairs of one (b, h), from each row's allowed interval.
+
+    Causal and sliding-window rows allow one interval of kv; a document row allows its
+    document's run of positions (document ids here form contiguous runs).
+    """
+    S = w.S
+    q = np.arange(S, dtype=np.int64)
+    lo = np.zeros(S, dtype=np.int64)
+    hi = np.full(S, S - 1, dtype=np.int64)
+    if w.mask_kind & (wl.MASK_CAUSAL | wl.MASK_SLIDING_WINDOW):
+        hi = np.minimum(hi, q)
+    if w.mask_kind & wl.MASK_SLIDING_WINDOW:
+        lo = np.maximum(lo, q - w.window + 1)
+    if w.mask_kind & wl.MASK_DOCUMENT:
+        if doc is None or np.any(np.diff(doc) < 0):
+            raise ValueError("document ids must form contiguous ascending runs")
+        starts = np.searchsorted(doc, doc, side="left")
+        ends = np.searchsorted(doc, doc, side="right") - 1
+        lo = np.maximum(lo, starts)
+        hi = np.minimum(hi, ends)
+    return int(np.clip(hi - lo + 1, 0, None).sum())
+
+
+def flops_per_step(w: wl.Workload, doc=None) -> float:
+    return 4.0 * w.D * live_positions_per_head(w, doc) * w.B * w.H
+
+
+# ---------------------------------------------------------------- environment helpers
+
+def read_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"bf16_tflops": float(d["bf16_tflops"]), "hbm_gbs": float(d["hbm_gbs"]),
+                "source": "measured"}
+    return {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("attn_fwd.cu", "sm100_ptx.cuh", "fa_internal.h"):
+        with open(os.path.join(ROOT, "block_sparse_masked_x128_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this kernel source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.reader.join(timeout=2)
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+
+def oracle_sample_rate(w: wl.Workload, q, k, v, doc, budget_s: float, rows_per_chunk: int = 256,
+                       seed: int = 0) -> dict:
+    """Time the float64 oracle on random query rows of the workload until budget_s elapses."""
+    import oracle
+    mm = oracle.make_mask_mod(w.mask_kind, window=w.window or None, document_id=doc)
+    sm = oracle.make_score_mod(w.score_kind, H=w.H, softcap=w.softcap or 30.0)
+    rng = np.random.default_rng(seed)
+    qn, kn, vn = (t.float().numpy() for t in (q, k, v))
+    live_row = _live_per_row(w, doc)
+    rows_done, live, t_total = 0, 0, 0.0
+    while t_total < budget_s:
+        b = int(rng.integers(0, w.B))
+        h = int(rng.integers(0, w.H))
+        rows = np.sort(rng.choice(w.S, size=min(rows_per_chunk, w.S), replace=False))
+        t0 = time.perf_counter()
+        oracle.attention(qn[b:b + 1, h:h + 1], kn[b:b + 1, h:h + 1], vn[b:b + 1, h:h + 1], mm,
+                         (lambda s, bb, hh, qi, ki, _h=h: sm(s, 0, _h, qi, ki)) if sm else None,
+                         scale=w.scale, rows=rows)
+        t_total += time.perf_counter() - t0
+        rows_done += len(rows)
+        live += int(live_row[rows].sum())
+    tflops = 4.0 * w.D * live / t_total / 1e12
+    return {"value": tflops, "rows": rows_done, "seconds": t_total, "live_positions": live}
+
+
+def _live_per_row(w, doc):
+    S = w.S
+    q = np.arange(S, dtype=np.int64)
+    lo = np.zeros(S, dtype=np.int64)
+    hi = np.full(S, S - 1, dtype=np.int64)
+    if w.mask_kind & (wl.MASK_CAUSAL | wl.MASK_SLIDING_WINDOW):
+        hi = np.minimum(hi, q)
+    if w.mask_kind & wl.MASK_SLIDING_WINDOW:
+        lo = np.maximum(lo, q - w.window + 1)
+    if w.mask_kind & wl.MASK_DOCUMENT:
+        lo = np.maximum(lo, np.searchsorted(doc, doc, side="left"))
+        hi = np.minimum(hi, np.searchsorted(doc, doc, side="right") - 1)
+    return np.clip(hi - lo + 1, 0, None)
+
+
+def cores_used() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        if blas:
+            return int(max(blas))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- arms
+
+def config_dict(w: wl.Workload, world: int) -> dict:
+    mask = []
+    if w.mask_kind & wl.MASK_CAUSAL:
+        mask.append("causal")
+    if w.mask_kind & wl.MASK_SLIDING_WINDOW:
+        mask.append(f"sliding_window(W={w.window})")
+    if w.mask_kind & wl.MASK_DOCUMENT:
+        mask.append(f"document({w.n_docs} seeded docs)")
+    score = []
+    if w.score_kind & wl.SCORE_SOFTCAP:
+        score.append(f"softcap({w.softcap:g})")
+    if w.score_kind & wl.SCORE_ALIBI:
+        score.append("alibi(2^(-8(h+1)/H))")
+    return {"workload": w.name, "B": w.B, "H": w.H, "Q_LEN": w.S, "KV_LEN": w.S, "head_dim": w.D,
+            "BLOCK_SIZE": 128, "mask_mod": " & ".join(mask) or "none",
+            "score_mod": " then ".join(score) or "none", "global_batch": w.B * world,
+            "seq_len": w.S, "parallelism": f"dp{world}",
+            "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every timed step"}
+
+
+def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
+    import torch
+    import block_sparse_masked_x128_b200 as fa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    q, k, v = wl.make_qkv(w, seed=w.seed + 1000 * rank)
+    doc = wl.make_doc_ids(w)
+    flops = flops_per_step(w, doc)
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    doc_d = torch.from_numpy(doc).to(dev) if doc is not None else None
+    stream = torch.cuda.current_stream()
+
+    # Mask build (once per shape; timed apart from the forward).
+    build_ms = []
+    bm = None
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        bm = fa.create_block_mask(w.mask_kind, None, None, w.S, w.S, window=w.window, doc_id=doc_d)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        build_ms.append(e0.elapsed_time(e1))
+    out = torch.empty_like(qd)
+    lse = torch.empty(w.B, w.H, w.S, device=dev, dtype=torch.float32)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap or 30.0,
+                          scale=w.scale, out=out, lse=lse)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd()
+    torch.cuda.synchronize()
+    if bm.device_status() != fa.FA_OK:
+        raise RuntimeError("a device-side wait timed out during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            fwd()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall0
+    barrier(world)
+    if bm.device_status() != fa.FA_OK:
+        raise RuntimeError("a device-side wait timed out during the timed steps")
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    t_fwd_ms = sum(per)
+    t_max_ms = max_over_ranks(t_fwd_ms, world, dev)
+    value = world * flops * args.steps / (t_max_ms * 1e-3) / 1e12
+    achieved = flops / (statistics.mean(per) * 1e-3) / 1e12
+
+    # End to end through the public API from pinned host buffers: H2D of q, k, v, the
+    # forward, D2H of out and lse, every step.
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        e2e_steps = max(3, min(args.steps, args.e2e_steps))
+        for _ in range(2):
+            qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+            fwd()
+            oh.copy_(out, non_blocking=True); lh.copy_(lse, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+            fwd()
+            oh.copy_(out, non_blocking=True); lh.copy_(lse, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        barrier(world)
+        e2e = {"value": world * flops * e2e_steps / (t_e2e * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in (q, k, v))),
+               "d2h_bytes_per_step": int(out.numel() * out.element_size() + lse.numel() * 4),
+               "steps": e2e_steps}
+
+    peaks = read_peaks()
+    traffic = recorded_traffic(w.name)
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": config_dict(w, world),
+        "pct_of_peak": 100.0 * value / world / peaks["bf16_tflops"],
+        "pct_of_nominal_2250": 100.0 * value / world / NOMINAL_BF16_TFLOPS,
+        "live_gflop_per_step": flops / 1e9,
+        "mask_build_ms": statistics.median(build_ms[1:]),
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": traffic, "peak_source": peaks["source"] + " bf16_tflops (burst)",
+                     "kernel": "attn_fwd_kernel"},
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": t_wall,
+    }
+    if e2e is not None:
+        res["e2e"] = e2e
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cb = oracle_sample_rate(w, q, k, v, doc, args.cpu_seconds)
+        res["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cores_used(),
+                               "kind": "oracle",
+                               "sample": f"{cb['rows']} random query rows of {w.name} "
+                                         f"({cb['seconds']:.1f} s of float64 oracle time)"}
+    return res
+
+
+def run_reference(args, w: wl.Workload, world: int, rank: int) -> dict:
+    """The oracle as the reference arm: each step is a bounded sample of query rows."""
+    q, k, v = wl.make_qkv(w)
+    doc = wl.make_doc_ids(w)
+    per_step = max(0.02, args.reference_budget_s / max(1, args.steps + args.warmup))
+    rows = 16
+    oracle_sample_rate(w, q, k, v, doc, 0.0, rows_per_chunk=rows)  # warm the imports
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, q, k, v, doc, 0.0, rows_per_chunk=rows)
+    t0 = time.perf_counter()
+    tot_live, tot_t, tot_rows = 0, 0.0, 0
+    for i in range(args.steps):
+        r = oracle_sample_rate(w, q, k, v, doc, 0.0, rows_per_chunk=rows, seed=i)
+        tot_live += r["live_positions"]
+        tot_t += r["seconds"]
+        tot_rows += r["rows"]
+        if time.perf_counter() - t0 > per_step * args.steps + 60:
+            break
+    value = 4.0 * w.D * tot_live / tot_t / 1e12
+    cores = cores_used()
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference", "config": config_dict(w, world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{tot_rows} query rows ({rows} per step) of {w.name}"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[x.name for x in wl.WORKLOADS])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-budget-s", type=float, default=60.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = wl.BY_NAME[args.workload]
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, w, world, rank)))
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        res = run_ours(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
