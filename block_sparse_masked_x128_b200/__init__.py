@@ -3,7 +3,7 @@
 A thin ctypes binding of the C ABI in ``include/fa_b200.h``.  It only marshals arguments:
 every step of the computation runs in the library's CUDA kernels.  PyTorch supplies device
 memory and streams.  There is no CPU fallback: importing this package fails loudly if the
-shared library has not been built (``python -m block_sparse_masked_x128_b200.build``).
+shared library has not been built (``python block_sparse_masked_x128_b200/build.py``).
 
 Low-level names mirror the C entry points (``fa_create_block_mask``, ``fa_forward``, ...).
 ``create_block_mask`` and ``flex_attention`` are the convenience forms named after the
@@ -19,7 +19,7 @@ from typing import Optional, Tuple
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libfa_b200.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
-        f"{_LIB_PATH} is missing: build it with `python -m block_sparse_masked_x128_b200.build`")
+        f"{_LIB_PATH} is missing: build it with `python block_sparse_masked_x128_b200/build.py`")
 _lib = ctypes.CDLL(_LIB_PATH)
 
 # ---------------------------------------------------------------- constants (fa_b200.h)
@@ -41,7 +41,8 @@ FA_DTYPE_F16 = 0
 FA_DTYPE_BF16 = 1
 
 EXPORTED = ("fa_create_block_mask", "fa_forward", "fa_block_mask_get", "fa_get_device_status",
-            "fa_destroy_block_mask", "fa_status_string", "fa_last_error_message")
+            "fa_destroy_block_mask", "fa_status_string", "fa_last_error_message",
+            "fa_create_block_mask_noalloc")
 
 
 class FaMaskParams(ctypes.Structure):
@@ -78,6 +79,11 @@ _lib.fa_forward.argtypes = [ctypes.POINTER(FaTensor), ctypes.POINTER(FaTensor), 
                             ctypes.c_void_p, ctypes.c_uint32, ctypes.POINTER(FaScoreParams),
                             ctypes.c_float, ctypes.POINTER(FaTensor), ctypes.c_void_p, ctypes.c_void_p]
 _lib.fa_forward.restype = _status
+_lib.fa_create_block_mask_noalloc.argtypes = [
+    ctypes.c_uint32, ctypes.POINTER(FaMaskParams), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+    ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+    ctypes.c_void_p]
+_lib.fa_create_block_mask_noalloc.restype = _status
 _lib.fa_block_mask_get.argtypes = [ctypes.c_void_p, ctypes.POINTER(FaBlockMaskInfo)]
 _lib.fa_block_mask_get.restype = _status
 _lib.fa_get_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
@@ -158,6 +164,18 @@ def fa_forward(q: FaTensor, k: FaTensor, v: FaTensor, block_mask: int, score_mod
                          ctypes.byref(params) if params is not None else None, scale, ctypes.byref(out),
                          lse_ptr, _stream_ptr(stream))
     _check(st, "fa_forward")
+
+
+def fa_create_block_mask_noalloc(mask_kind: int, params: Optional[FaMaskParams], B: int, H: int,
+                                 Q_LEN: int, KV_LEN: int, BLOCK_SIZE: int, kv_num_blocks: int,
+                                 kv_indices: int, full_kv_num_blocks: int, full_kv_indices: int,
+                                 stream=None) -> None:
+    """Call fa_create_block_mask_noalloc: build the four lists into caller-owned device buffers
+    (pointers as integers) without any device allocation by the library."""
+    st = _lib.fa_create_block_mask_noalloc(mask_kind, ctypes.byref(params) if params is not None else None,
+                                           B, H, Q_LEN, KV_LEN, BLOCK_SIZE, kv_num_blocks, kv_indices,
+                                           full_kv_num_blocks, full_kv_indices, _stream_ptr(stream))
+    _check(st, "fa_create_block_mask_noalloc")
 
 
 def fa_block_mask_get(block_mask: int) -> FaBlockMaskInfo:

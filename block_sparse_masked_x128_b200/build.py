@@ -1,6 +1,8 @@
 """Build the sm_100a shared library in-tree: block_sparse_masked_x128_b200/_lib/libfa_b200.so.
 
-    python -m block_sparse_masked_x128_b200.build [--verbose]
+    python block_sparse_masked_x128_b200/build.py [--verbose] [--ptxas-info] [--force]
+
+(Run it as a file, not as a package module: importing the package loads the library.)
 
 Each .cu file is compiled to an object in parallel (nvcc cross-compiles for sm_100a without
 a GPU), then linked into one shared library exporting the C ABI of include/fa_b200.h.
@@ -8,6 +10,7 @@ Objects are rebuilt only when a source or header is newer.  `--ptxas-info` print
 registers and shared memory of every kernel (nvcc -Xptxas -v).
 """
 from __future__ import annotations
+
 
 import argparse
 import concurrent.futures as cf
@@ -23,7 +26,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libfa_b200.so")
-SOURCES = ["api.cu", "mask_builder.cu", "attn_fwd.cu"]
+SOURCES = ["api.cu", "mask_builder.cu", "attn_fwd.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -108,6 +108,13 @@ fa_status_t check_tensor(const fa_tensor_t* t, const char* name) {
 
 }  // namespace
 
+namespace fa {
+fa_status_t record_error(fa_status_t status, const char* message) {
+    return fail(status, "%s", message);
+}
+fa_status_t record_ok() { return ok(); }
+}  // namespace fa
+
 extern "C" {
 
 const char* fa_status_string(fa_status_t s) {

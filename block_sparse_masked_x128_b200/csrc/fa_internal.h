@@ -61,6 +61,16 @@ cudaError_t launch_mask_build(const MaskSpec& spec, int separate_full, int maskB
                               int32_t* sched_cost, int32_t* sched_entries, int32_t* sched_order,
                               cudaStream_t stream);
 
+// Only the tile classification and list compaction of launch_mask_build (no schedule),
+// with the per-block document statistics at `doc_stats`.
+cudaError_t launch_mask_lists(const MaskSpec& spec, int separate_full, int maskBH,
+                              int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
+                              int32_t* full_idx, int32_t* doc_stats, cudaStream_t stream);
+
+// Set the calling thread's last-error message (read by fa_last_error_message).
+fa_status_t record_error(fa_status_t status, const char* message);
+fa_status_t record_ok();
+
 cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, bool has_score,
                             const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             int grid, cudaStream_t stream);

@@ -259,6 +259,23 @@ __global__ void __launch_bounds__(1024) lpt_order_kernel(int NP, const int32_t* 
 
 }  // namespace
 
+cudaError_t launch_mask_lists(const MaskSpec& spec, int separate_full, int maskBH,
+                              int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
+                              int32_t* full_idx, int32_t* doc_stats, cudaStream_t stream) {
+    if (spec.kind & FA_MASK_DOCUMENT) {
+        const int nblk = spec.QB > spec.KVB ? spec.QB : spec.KVB;
+        doc_block_stats_kernel<<<nblk, kThreads, 0, stream>>>(spec.doc, spec.KV_LEN, nblk,
+                                                              doc_stats);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    MaskSpec s = spec;
+    s.doc_stats = doc_stats;
+    classify_compact_kernel<<<dim3(spec.QB, maskBH), kThreads, 0, stream>>>(
+        s, separate_full, kv_num, kv_idx, full_num, full_idx);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_mask_build(const MaskSpec& spec, int separate_full, int maskBH, int NP,
                               int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
                               int32_t* full_idx, int32_t* doc_stats, int32_t* sched_count,

@@ -155,6 +155,39 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
                        const fa_score_params_t* params, float scale,
                        fa_tensor_t* out, float* lse, void* stream);
 
+/*
+ * fa_create_block_mask_noalloc -- the block-mask build of fa_create_block_mask, writing into
+ * caller-owned lists and allocating no device memory.  (The pages have no counterpart: it
+ * exists for callers that cannot let a library allocate.)
+ *
+ * Who needs it: code running inside a framework whose caching allocator or arena already
+ * owns the GPU's memory (a cudaMalloc behind its back escapes its accounting and can fail
+ * once the pool holds most of HBM), plugins of inference runtimes whose enqueue path must
+ * not allocate, and real-time deployments that forbid allocation after start-up; cudaMalloc
+ * can also synchronise the device, which latency-critical callers cannot afford.
+ *
+ * Arguments are those of fa_create_block_mask, except that the four lists are written to
+ * caller-owned device buffers laid out as in fa_block_mask_info_t:
+ *   kv_num_blocks, full_kv_num_blocks   int32 [B'][H'][q_blocks]
+ *   kv_indices, full_kv_indices         int32 [B'][H'][q_blocks][kv_blocks]
+ * with B' = max(B, 1), H' = max(H, 1), q_blocks = ceil(Q_LEN/128), kv_blocks =
+ * ceil(KV_LEN/128); every element is written.  params->doc_id is read in place (not copied)
+ * and must stay valid until the stream has run the build.
+ *
+ * Limit and scratch: Q_LEN and KV_LEN may not exceed 4096 blocks (524288 positions); larger
+ * requests return FA_ERR_UNSUPPORTED.  Document statistics go to a fixed 48 KiB
+ * __device__ array that every GPU loading this library holds until exit.  All calls share
+ * it (it keeps the last call's contents; each call writes every entry it reads), so calls
+ * whose work overlaps on the GPU -- e.g. on two streams -- race.  The first call on a
+ * device looks up the array's address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.
+ */
+fa_status_t fa_create_block_mask_noalloc(uint32_t mask_kind, const fa_mask_params_t* params,
+                                         int32_t B, int32_t H, int32_t Q_LEN, int32_t KV_LEN,
+                                         int32_t BLOCK_SIZE, int32_t* kv_num_blocks,
+                                         int32_t* kv_indices, int32_t* full_kv_num_blocks,
+                                         int32_t* full_kv_indices, void* stream);
+
 /* Fill `info` with the mask's extents and device pointers.  FA_ERR_INVALID_ARG on NULL. */
 fa_status_t fa_block_mask_get(const fa_block_mask_t* block_mask, fa_block_mask_info_t* info);
 

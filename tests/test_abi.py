@@ -9,10 +9,18 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+def _build_module():
+    import importlib.util
+    path = os.path.join(ROOT, "block_sparse_masked_x128_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_fa_b200_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
 @pytest.fixture(scope="module")
 def fa():
-    from block_sparse_masked_x128_b200 import build
-    build.build()
+    _build_module().build()
     import block_sparse_masked_x128_b200 as fa
     return fa
 
@@ -38,8 +46,7 @@ def test_library_exports_every_declared_symbol(fa):
 
 
 def test_library_is_built_for_sm100a_only():
-    from block_sparse_masked_x128_b200 import build
-    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert _build_module().ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
 def test_status_strings(fa):
