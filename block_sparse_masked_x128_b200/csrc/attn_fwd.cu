@@ -70,6 +70,15 @@ struct Unit {
     const int32_t* entries;
 };
 
+// The k-th unit of this CTA.  Units are in descending-cost order; rounds of gridDim.x
+// units are dealt alternately forwards and backwards over the CTAs ("snake" order), which
+// keeps the per-CTA sums of a longest-first list close to equal.
+__device__ __forceinline__ int unit_of_round(int k) {
+    const int G = (int)gridDim.x;
+    const int slot = (k & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+    return k * G + slot;
+}
+
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     const int BH = p.B * p.H;
     const int r = u / BH, bh = u - r * BH;
@@ -147,7 +156,9 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
     }
     uint32_t kv_pos = 0, q_iter = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    for (int k = 0; ok; ++k) {
+        const int u = unit_of_round(k);
+        if (u >= p.n_units) break;
         const Unit un = decode_unit(p, u);
         if (un.E == 0) continue;
         if (!wait(kBarQEmpty, (q_iter & 1u) ^ 1u)) { ok = false; break; }
@@ -238,7 +249,9 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
     uint32_t kv_pos = 0, q_iter = 0;
     uint32_t pf_cnt[2] = {0u, 0u}, of_cnt[2] = {0u, 0u};
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    for (int k = 0; ok; ++k) {
+        const int u = unit_of_round(k);
+        if (u >= p.n_units) break;
         const Unit un = decode_unit(p, u);
         if (un.E == 0) continue;
         int nl[2];
@@ -353,7 +366,9 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
     const bool has_alibi = SCORE && (p.score_kind & FA_SCORE_ALIBI);
 
     uint32_t sf_cnt = 0, of_cnt = 0;
-    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    for (int k = 0;; ++k) {
+        const int u = unit_of_round(k);
+        if (u >= p.n_units) break;
         const Unit un = decode_unit(p, u);
         const int qblk = 2 * un.pair + t;
         if (qblk >= p.QB) continue;
@@ -391,26 +406,44 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             if (!wait(kBarSFull + t, sf_cnt & 1u)) { ok = false; break; }
             ++sf_cnt;
             tc_fence_after();
-            uint32_t sr[4][32];
+            // S row of this thread: 128 fp32 scores held as 64 pairs.
+            float2 x[64];
+            {
+                uint32_t sr[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, sr[c]);
-            tmem_ld_wait();
+                for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, sr[c]);
+                tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 4; ++c) reg_fence<32>(sr[c]);
-            float x[128];
+                for (int c = 0; c < 4; ++c) reg_fence<32>(sr[c]);
 #pragma unroll
-            for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c >> 5][c & 31]);
+                for (int i = 0; i < 64; ++i)
+                    x[i] = make_float2(__uint_as_float(sr[i >> 4][(2 * i) & 31]),
+                                       __uint_as_float(sr[i >> 4][(2 * i + 1) & 31]));
+            }
             const int kv0 = j * kBlock;
             if constexpr (SCORE) {
                 // score_mod on every position of the tile, in log2 units; masked
                 // positions are set to -inf afterwards (the mask decides liveness).
-                const float fb = (float)(kv0 - q);
+                const float2 inv2 = make_float2(p.inv_softcap_scale, p.inv_softcap_scale);
+                const float2 cap2 = make_float2(p.softcap_log2, p.softcap_log2);
+                const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+                const float2 sl2 = make_float2(slope_log2, slope_log2);
+                const float2 two = make_float2(2.f, 2.f);
+                float2 pos = make_float2((float)(kv0 - q), (float)(kv0 - q + 1));
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    float y = has_softcap ? p.softcap_log2 * tanh_approx(x[c] * p.inv_softcap_scale)
-                                          : x[c] * p.scale_log2;
-                    if (has_alibi) y = fmaf(slope_log2, fb + (float)c, y);
-                    x[c] = y;
+                for (int i = 0; i < 64; ++i) {
+                    float2 y;
+                    if (has_softcap) {
+                        const float2 a = __fmul2_rn(x[i], inv2);
+                        y = __fmul2_rn(cap2, make_float2(tanh_approx(a.x), tanh_approx(a.y)));
+                    } else {
+                        y = __fmul2_rn(x[i], sc2);
+                    }
+                    if (has_alibi) {
+                        y = __ffma2_rn(sl2, pos, y);
+                        pos = __fadd2_rn(pos, two);
+                    }
+                    x[i] = y;
                 }
             }
             if (!full) {
@@ -424,72 +457,75 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                     for (int c4 = 0; c4 < 32; ++c4) {
                         const int4 d4 = __ldg(dk + c4);
                         const int c = 4 * c4;
-                        if (!(c + 0 >= lo && c + 0 <= hi && d4.x == dq)) x[c + 0] = -INFINITY;
-                        if (!(c + 1 >= lo && c + 1 <= hi && d4.y == dq)) x[c + 1] = -INFINITY;
-                        if (!(c + 2 >= lo && c + 2 <= hi && d4.z == dq)) x[c + 2] = -INFINITY;
-                        if (!(c + 3 >= lo && c + 3 <= hi && d4.w == dq)) x[c + 3] = -INFINITY;
+                        if (!(c + 0 >= lo && c + 0 <= hi && d4.x == dq)) x[2 * c4].x = -INFINITY;
+                        if (!(c + 1 >= lo && c + 1 <= hi && d4.y == dq)) x[2 * c4].y = -INFINITY;
+                        if (!(c + 2 >= lo && c + 2 <= hi && d4.z == dq)) x[2 * c4 + 1].x = -INFINITY;
+                        if (!(c + 3 >= lo && c + 3 <= hi && d4.w == dq)) x[2 * c4 + 1].y = -INFINITY;
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if (c < lo || c > hi) x[c] = -INFINITY;
+                    for (int i = 0; i < 64; ++i) {
+                        if (2 * i < lo || 2 * i > hi) x[i].x = -INFINITY;
+                        if (2 * i + 1 < lo || 2 * i + 1 > hi) x[i].y = -INFINITY;
+                    }
                 }
             }
-            float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+            // Row max with three-input max: four independent chains over quarters.
+            float mc[4];
 #pragma unroll
-            for (int c = 4; c < 128; c += 4) {
-                mx0 = fmaxf(mx0, x[c]);
-                mx1 = fmaxf(mx1, x[c + 1]);
-                mx2 = fmaxf(mx2, x[c + 2]);
-                mx3 = fmaxf(mx3, x[c + 3]);
-            }
-            float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            for (int c = 0; c < 4; ++c) mc[c] = fmaxf(x[16 * c].x, x[16 * c].y);
+#pragma unroll
+            for (int i = 1; i < 16; ++i)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) mc[c] = max3(mc[c], x[16 * c + i].x, x[16 * c + i].y);
+            float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
             if constexpr (!SCORE) mt *= p.scale_log2;
             const float m_new = fmaxf(m, mt);
             const bool need = m_new > m + kRescaleThreshold;
-            if (__any_sync(kFullMask, need)) {
-                const float alpha = need ? ex2_approx(m - m_new) : 1.0f;
-                if (done > 0) {
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld_32x32b_x32(tO + c * 32, o);
-                        tmem_ld_wait();
-                        reg_fence<32>(o);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st_32x32b_x32(tO + c * 32, o);
-                    }
-                    tmem_st_wait();
-                }
-                if (need) {
-                    l *= alpha;
-                    m = m_new;
-                }
+            const bool any_need = __any_sync(kFullMask, need);
+            float alpha = 1.0f;
+            if (need) {
+                alpha = ex2_approx(m - m_new);  // m = -inf gives 0 (l and O are empty then)
+                m = m_new;
             }
             const float base = (m == -INFINITY) ? 0.f : m;
-            float rs0 = 0.f, rs1 = 0.f;
+            // P = 2^(x - base) in 16-bit pairs, written over S in four chunks.
+            float2 rs = make_float2(0.f, 0.f);
+            const float2 nb2 = make_float2(-base, -base);
+            const float2 k2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32];
+            for (int chunk = 0; chunk < 4; ++chunk) {
+                uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int c = half * 64 + 2 * i;
-                    float p0, p1;
-                    if constexpr (SCORE) {
-                        p0 = ex2_approx(x[c] - base);
-                        p1 = ex2_approx(x[c + 1] - base);
-                    } else {
-                        p0 = ex2_approx(fmaf(x[c], p.scale_log2, -base));
-                        p1 = ex2_approx(fmaf(x[c + 1], p.scale_log2, -base));
-                    }
-                    rs0 += p0;
-                    rs1 += p1;
-                    pk[i] = pack2<BF16>(p0, p1);
+                for (int i = 0; i < 16; ++i) {
+                    const float2 a = SCORE ? __fadd2_rn(x[chunk * 16 + i], nb2)
+                                           : __ffma2_rn(x[chunk * 16 + i], k2, nb2);
+                    const float2 pe = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+                    rs = __fadd2_rn(rs, pe);
+                    pk[i] = pack2<BF16>(pe.x, pe.y);
                 }
-                tmem_st_32x32b_x32(tS + half * 32, pk);
+                tmem_st_32x32b_x16(tS + chunk * 16, pk);
             }
-            l += rs0 + rs1;
+            l = fmaf(l, alpha, rs.x + rs.y);
+            if (any_need && done > 0) {
+                // Rescale O only now, after S has left the registers.
+                const float2 al2 = make_float2(alpha, alpha);
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld_32x32b_x32(tO + c * 32, o);
+                    tmem_ld_wait();
+                    reg_fence<32>(o);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 v = __fmul2_rn(
+                            make_float2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), al2);
+                        o[2 * i] = __float_as_uint(v.x);
+                        o[2 * i + 1] = __float_as_uint(v.y);
+                    }
+                    tmem_st_32x32b_x32(tO + c * 32, o);
+                }
+            }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(bar(kBarPFull + t));
@@ -568,11 +604,18 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        producer_role<D>(p, &tmq, &tmk, &tmv, sbase, bars, abort_flag);
-    } else if (warp == 1) {
-        mma_role<D, BF16>(p, sbase, bars, tmem, abort_flag);
-    } else if (warp >= 4) {
+    // Registers: the TMA/MMA warpgroup needs few, the softmax warpgroups hold a 128-wide
+    // score row each.  4 warps x 64 + 8 warps x 216 fits the 384 x 168 launched.  Each
+    // role runs inside the branch of its own budget.
+    if (warp < 4) {
+        regs_dec<64>();
+        if (warp == 0) {
+            producer_role<D>(p, &tmq, &tmk, &tmv, sbase, bars, abort_flag);
+        } else if (warp == 1) {
+            mma_role<D, BF16>(p, sbase, bars, tmem, abort_flag);
+        }
+    } else {
+        regs_inc<216>();
         softmax_role<D, BF16, SCORE>(p, (warp - 4) >> 2, bars, tmem, abort_flag);
     }
     tc_fence_before();
