@@ -26,6 +26,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libfa_b200.so")
+TRACE_LIB = os.path.join(LIBDIR, "libfa_b200_trace.so")
 SOURCES = ["api.cu", "mask_builder.cu", "attn_fwd.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -37,11 +38,13 @@ def _nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _flags(ptxas_info: bool) -> list:
+def _flags(ptxas_info: bool, trace: bool = False) -> list:
     f = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
                 "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]
     if ptxas_info:
         f += ["-Xptxas", "-v"]
+    if trace:
+        f += ["-DFA_TRACE"]
     return f
 
 
@@ -50,8 +53,8 @@ def _headers() -> list:
     return hs + [os.path.join(INCLUDE, h) for h in os.listdir(INCLUDE) if h.endswith(".h")]
 
 
-def _compile(src: str, flags: list, force: bool) -> tuple:
-    obj = os.path.join(BUILD, os.path.splitext(src)[0] + ".o")
+def _compile(src: str, flags: list, force: bool, build_dir: str = BUILD) -> tuple:
+    obj = os.path.join(build_dir, os.path.splitext(src)[0] + ".o")
     srcp = os.path.join(CSRC, src)
     newest = max(os.path.getmtime(p) for p in [srcp] + _headers())
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= newest:
@@ -63,24 +66,28 @@ def _compile(src: str, flags: list, force: bool) -> tuple:
     return obj, r.stdout + r.stderr
 
 
-def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False,
+          trace: bool = False) -> str:
+    """Build the library; with trace=True build the phase-tracing variant instead."""
+    build_dir = os.path.join(BUILD, "trace") if trace else BUILD
+    lib = TRACE_LIB if trace else LIB
+    os.makedirs(build_dir, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
-    flags = _flags(ptxas_info)
+    flags = _flags(ptxas_info, trace)
     with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        results = list(ex.map(lambda s: _compile(s, flags, force or ptxas_info), SOURCES))
+        results = list(ex.map(lambda s: _compile(s, flags, force or ptxas_info, build_dir), SOURCES))
     objs = [o for o, _ in results]
     if verbose or ptxas_info:
         for _, log in results:
             if log:
                 print(log)
     newest_obj = max(os.path.getmtime(o) for o in objs)
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < newest_obj:
-        cmd = [_nvcc()] + ARCH + ["-shared", "-o", LIB] + objs + ["-lcudart_static", "-ldl", "-lrt", "-lpthread"]
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < newest_obj:
+        cmd = [_nvcc()] + ARCH + ["-shared", "-o", lib] + objs + ["-lcudart_static", "-ldl", "-lrt", "-lpthread"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 def main(argv=None) -> int:
@@ -88,8 +95,9 @@ def main(argv=None) -> int:
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true")
     ap.add_argument("--force", action="store_true")
+    ap.add_argument("--trace", action="store_true", help="build the phase-tracing variant")
     a = ap.parse_args(argv)
-    print(build(a.verbose, a.ptxas_info, a.force))
+    print(build(a.verbose, a.ptxas_info, a.force, a.trace))
     return 0
 
 

@@ -28,7 +28,14 @@
 #include <cfloat>
 
 #include "fa_internal.h"
+#include "fa_trace.cuh"
 #include "sm100_ptx.cuh"
+
+#ifdef FA_TRACE
+extern "C" int fa_debug_set_trace_buffer(void* device_ptr) {
+    return (int)cudaMemcpyToSymbol(g_fa_trace, &device_ptr, sizeof(device_ptr));
+}
+#endif
 
 namespace fa {
 namespace {
@@ -143,35 +150,36 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
                               const CUtensorMap* tmv, uint32_t sbase, uint32_t bars,
                               volatile int* abort_flag) {
     using C = Cfg<D>;
-    const int lane = threadIdx.x & 31;
     const uint32_t sQ = sbase, sKV = sbase + 2 * C::kTileBytes;
     auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
     auto wait = [&](int i, uint32_t par) {
         return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
     };
-    if (lane == 0) {
+    const uint32_t leader = elect_one_lane();
+    if (leader) {
         tma_prefetch_desc(tmq);
         tma_prefetch_desc(tmk);
         tma_prefetch_desc(tmv);
     }
+    __syncwarp();
     uint32_t kv_pos = 0, q_iter = 0;
     bool ok = true;
+    int tn = 0;
+    (void)tn;
     for (int k = 0; ok; ++k) {
         const int u = unit_of_round(k);
         if (u >= p.n_units) break;
         const Unit un = decode_unit(p, u);
         if (un.E == 0) continue;
+        FA_TRACE_EV(0, tn, 40);
         if (!wait(kBarQEmpty, (q_iter & 1u) ^ 1u)) { ok = false; break; }
         const int q0 = 2 * un.pair;
         const int nq = (q0 + 1 < p.QB) ? 2 : 1;
-        if (lane == 0) {
-            mbar_arrive_expect_tx(bar(kBarQFull), (uint32_t)(nq * C::kTileBytes));
-            for (int t = 0; t < nq; ++t)
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_4d(sQ + t * C::kTileBytes + c * 16384, tmq, bar(kBarQFull), c * 64,
-                                (q0 + t) * kBlock, un.h, un.b);
-        }
-        __syncwarp();
+        mbar_arrive_expect_tx_if(leader, bar(kBarQFull), (uint32_t)(nq * C::kTileBytes));
+        for (int t = 0; t < nq; ++t)
+            for (int c = 0; c < C::kChunks; ++c)
+                tma_load_4d_if(leader, sQ + t * C::kTileBytes + c * 16384, tmq, bar(kBarQFull),
+                               c * 64, (q0 + t) * kBlock, un.h, un.b);
         ++q_iter;
         EntryReader er;
         er.init(un.entries, un.E);
@@ -180,15 +188,14 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
             for (int which = 0; which < 2; ++which) {
                 const int s = (int)(kv_pos % C::kStages);
                 const uint32_t ph = (kv_pos / C::kStages) & 1u;
+                FA_TRACE_EV(0, tn, 30 + which);
                 if (!wait(C::kBarSlotEmpty + s, ph ^ 1u)) { ok = false; break; }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(bar(kBarSlotFull + s), (uint32_t)C::kTileBytes);
-                    const CUtensorMap* tm = which ? tmv : tmk;
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_4d(sKV + s * C::kTileBytes + c * 16384, tm, bar(kBarSlotFull + s),
-                                    c * 64, j * kBlock, un.h, un.b);
-                }
-                __syncwarp();
+                FA_TRACE_EV(0, tn, 32 + which);
+                mbar_arrive_expect_tx_if(leader, bar(kBarSlotFull + s), (uint32_t)C::kTileBytes);
+                const CUtensorMap* tm = which ? tmv : tmk;
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_4d_if(leader, sKV + s * C::kTileBytes + c * 16384, tm,
+                                   bar(kBarSlotFull + s), c * 64, j * kBlock, un.h, un.b);
                 ++kv_pos;
             }
         }
@@ -210,7 +217,7 @@ template <int D, bool BF16>
 __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          volatile int* abort_flag) {
     using C = Cfg<D>;
-    const int lane = threadIdx.x & 31;
+    const uint32_t leader = elect_one_lane();
     const uint32_t sQ = sbase, sKV = sbase + 2 * C::kTileBytes;
     constexpr uint32_t kIdescQK = make_idesc_f16(BF16, 128, 128, false);
     constexpr uint32_t kIdescPV = make_idesc_f16(BF16, 128, D, true);
@@ -224,12 +231,13 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
     // next 16 KB box.
     auto issue_qk = [&](int t, int slot) {
         const uint32_t d = tmem + C::colS(t);
-        const uint32_t qa = sQ + t * C::kTileBytes, ka = sKV + slot * C::kTileBytes;
+        const uint64_t qd = make_sdesc_sw128(sQ + t * C::kTileBytes, 16, 1024);
+        const uint64_t kd = make_sdesc_sw128(sKV + slot * C::kTileBytes, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32);
-            mma_ss(d, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
-                   kIdescQK, kk > 0 ? 1u : 0u);
+            // Start-address field counts 16-byte units: add the byte offset >> 4.
+            const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_ss_if(leader, d, qd + off, kd + off, kIdescQK, kk > 0 ? 1u : 0u);
         }
     };
     // O_t += P_t V: M = 128, N = D, K = 128 keys in steps of 16.  P_t comes from TMEM
@@ -238,17 +246,19 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
     auto issue_pv = [&](int t, int slot, bool accumulate) {
         const uint32_t d = tmem + C::colO(t);
         const uint32_t pa = tmem + C::colS(t);
-        const uint32_t va = sKV + slot * C::kTileBytes;
+        const uint64_t vd = make_sdesc_sw128(sKV + slot * C::kTileBytes, 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk) {
-            mma_ts(d, pa + (uint32_t)(kk * 8), make_sdesc_sw128(va + kk * 2048, 16384, 1024),
-                   kIdescPV, (kk > 0 || accumulate) ? 1u : 0u);
+            mma_ts_if(leader, d, pa + (uint32_t)(kk * 8), vd + (uint64_t)((kk * 2048) >> 4), kIdescPV,
+                      (kk > 0 || accumulate) ? 1u : 0u);
         }
     };
 
     uint32_t kv_pos = 0, q_iter = 0;
     uint32_t pf_cnt[2] = {0u, 0u}, of_cnt[2] = {0u, 0u};
     bool ok = true;
+    int tn = 0;
+    (void)tn;
     for (int k = 0; ok; ++k) {
         const int u = unit_of_round(k);
         if (u >= p.n_units) break;
@@ -270,57 +280,50 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
             const int s = (int)(pos % C::kStages);
             if (!wait(kBarSlotFull + s, (pos / C::kStages) & 1u)) { ok = false; break; }
             tc_fence_after();
-            if (lane == 0) {
-                for (int t = 0; t < 2; ++t)
-                    if (code & (t ? kLive1 : kLive0)) {
-                        issue_qk(t, s);
-                        tc_commit(bar(kBarSFull + t));
-                    }
-                tc_commit(bar(C::kBarSlotEmpty + s));
-                if (un.E == 1) tc_commit(bar(kBarQEmpty));
-            }
-            __syncwarp();
+            for (int t = 0; t < 2; ++t)
+                if (code & (t ? kLive1 : kLive0)) {
+                    issue_qk(t, s);
+                    tc_commit_if(leader, bar(kBarSFull + t));
+                }
+            tc_commit_if(leader, bar(C::kBarSlotEmpty + s));
+            if (un.E == 1) tc_commit_if(leader, bar(kBarQEmpty));
         }
         for (int e = 0; e < un.E; ++e) {
             const bool has_next = e + 1 < un.E;
             const int next = has_next ? er.get(e + 1) : 0;
             const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u, kpos = vpos + 1u;
             const int vs = (int)(vpos % C::kStages), ks = (int)(kpos % C::kStages);
+            FA_TRACE_EV(1, tn, 22);
             if (!wait(kBarSlotFull + vs, (vpos / C::kStages) & 1u)) { ok = false; break; }
             if (has_next && !wait(kBarSlotFull + ks, (kpos / C::kStages) & 1u)) { ok = false; break; }
+            FA_TRACE_EV(1, tn, 23);
             tc_fence_after();
             for (int t = 0; t < 2; ++t) {
                 if (code & (t ? kLive1 : kLive0)) {
+                    FA_TRACE_EV(1, tn, 16 + t);
                     if (!wait(kBarPFull + t, pf_cnt[t] & 1u)) { ok = false; break; }
+                    FA_TRACE_EV(1, tn, 18 + t);
                     ++pf_cnt[t];
                     if (ndone[t] == 0 && !wait(kBarOFree + t, (of_cnt[t] & 1u) ^ 1u)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    if (lane == 0) {
-                        issue_pv(t, vs, ndone[t] > 0);
-                        if (ndone[t] + 1 == nl[t]) tc_commit(bar(kBarOFull + t));
-                    }
+                    issue_pv(t, vs, ndone[t] > 0);
+                    if (ndone[t] + 1 == nl[t]) tc_commit_if(leader, bar(kBarOFull + t));
                     ++ndone[t];
                 }
                 if (next & (t ? kLive1 : kLive0)) {
-                    if (lane == 0) {
-                        issue_qk(t, ks);
-                        tc_commit(bar(kBarSFull + t));
-                    }
+                    issue_qk(t, ks);
+                    tc_commit_if(leader, bar(kBarSFull + t));
                 }
-                __syncwarp();
             }
             if (!ok) break;
-            if (lane == 0) {
-                tc_commit(bar(C::kBarSlotEmpty + vs));
-                if (has_next) {
-                    tc_commit(bar(C::kBarSlotEmpty + ks));
-                    if (e + 2 == un.E) tc_commit(bar(kBarQEmpty));
-                }
+            tc_commit_if(leader, bar(C::kBarSlotEmpty + vs));
+            if (has_next) {
+                tc_commit_if(leader, bar(C::kBarSlotEmpty + ks));
+                if (e + 2 == un.E) tc_commit_if(leader, bar(kBarQEmpty));
             }
-            __syncwarp();
             code = next;
         }
         if (!ok) break;
@@ -329,8 +332,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
     }
     if (!ok) {
         // Wait for every MMA already issued before the CTA can release TMEM.
-        if (lane == 0) tc_commit(bar(kBarDrain));
-        __syncwarp();
+        tc_commit_if(leader, bar(kBarDrain));
         drain_wait(bar(kBarDrain), 0u);
     }
 }
@@ -366,6 +368,10 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
     const bool has_alibi = SCORE && (p.score_kind & FA_SCORE_ALIBI);
 
     uint32_t sf_cnt = 0, of_cnt = 0;
+    const int tslot = 2 + (int)(threadIdx.x >> 5) - 4;  // one trace slot per softmax warp
+    int tn = 0;
+    (void)tslot;
+    (void)tn;
     for (int k = 0;; ++k) {
         const int u = unit_of_round(k);
         if (u >= p.n_units) break;
@@ -403,7 +409,9 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             if (!(code & live_bit)) continue;
             const int j = code & 0xFFFF;
             const bool full = (code & full_bit) != 0;
+            FA_TRACE_EV(tslot, tn, 1);
             if (!wait(kBarSFull + t, sf_cnt & 1u)) { ok = false; break; }
+            FA_TRACE_EV(tslot, tn, 2);
             ++sf_cnt;
             tc_fence_after();
             // S row of this thread: 128 fp32 scores held as 64 pairs.
@@ -420,6 +428,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                     x[i] = make_float2(__uint_as_float(sr[i >> 4][(2 * i) & 31]),
                                        __uint_as_float(sr[i >> 4][(2 * i + 1) & 31]));
             }
+            FA_TRACE_EV(tslot, tn, 3);
             const int kv0 = j * kBlock;
             if constexpr (SCORE) {
                 // score_mod on every position of the tile, in log2 units; masked
@@ -481,6 +490,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
             if constexpr (!SCORE) mt *= p.scale_log2;
             const float m_new = fmaxf(m, mt);
+            FA_TRACE_EV(tslot, tn, 4);
             const bool need = m_new > m + kRescaleThreshold;
             const bool any_need = __any_sync(kFullMask, need);
             float alpha = 1.0f;
@@ -507,6 +517,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                 tmem_st_32x32b_x16(tS + chunk * 16, pk);
             }
             l = fmaf(l, alpha, rs.x + rs.y);
+            FA_TRACE_EV(tslot, tn, 5);
             if (any_need && done > 0) {
                 // Rescale O only now, after S has left the registers.
                 const float2 al2 = make_float2(alpha, alpha);
@@ -529,10 +540,12 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(bar(kBarPFull + t));
+            FA_TRACE_EV(tslot, tn, 6);
             ++done;
         }
         if (!ok) return;
         // Epilogue: O / l in the output dtype, and the natural-log lse.
+        FA_TRACE_EV(tslot, tn, 7);
         if (!wait(kBarOFull + t, of_cnt & 1u)) return;
         ++of_cnt;
         tc_fence_after();
@@ -559,6 +572,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                 (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
         tc_fence_before();
         mbar_arrive(bar(kBarOFree + t));
+        FA_TRACE_EV(tslot, tn, 8);
     }
 }
 
@@ -605,17 +619,17 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
     const uint32_t tmem = *tmem_slot;
 
     // Registers: the TMA/MMA warpgroup needs few, the softmax warpgroups hold a 128-wide
-    // score row each.  4 warps x 64 + 8 warps x 216 fits the 384 x 168 launched.  Each
+    // score row each.  4 warps x 80 + 8 warps x 208 fits the 384 x 168 launched.  Each
     // role runs inside the branch of its own budget.
     if (warp < 4) {
-        regs_dec<64>();
+        regs_dec<80>();
         if (warp == 0) {
             producer_role<D>(p, &tmq, &tmk, &tmv, sbase, bars, abort_flag);
         } else if (warp == 1) {
             mma_role<D, BF16>(p, sbase, bars, tmem, abort_flag);
         }
     } else {
-        regs_inc<216>();
+        regs_inc<208>();
         softmax_role<D, BF16, SCORE>(p, (warp - 4) >> 2, bars, tmem, abort_flag);
     }
     tc_fence_before();
