@@ -366,7 +366,7 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
     const int nsm = sm_count(dev);
     if (nsm <= 0) return fail(FA_ERR_CUDA, "could not read the SM count");
     const int grid = p.n_units < nsm ? p.n_units : nsm;
-    e = fa::launch_attn_fwd(p, (int)q->D, q->dtype == FA_DTYPE_BF16, score_mod_kind != 0, tq, tk, tv,
+    e = fa::launch_attn_fwd(p, (int)q->D, q->dtype == FA_DTYPE_BF16, (int)score_mod_kind, tq, tk, tv,
                             grid, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");
     return ok();

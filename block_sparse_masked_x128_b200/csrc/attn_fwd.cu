@@ -54,8 +54,10 @@ enum : int {
     kBarPFull = 4,    // + tile
     kBarOFull = 6,    // + tile
     kBarOFree = 8,    // + tile
-    kBarDrain = 10,
-    kBarSlotFull = 11 // + stage, then slot-empty barriers follow
+    kBarSFree = 10,   // + tile: softmax has S in registers (separate-P layout only)
+    kBarPVDone = 12,  // + tile: the tile's last P.V has completed (separate-P layout only)
+    kBarDrain = 14,
+    kBarSlotFull = 15 // + stage, then slot-empty barriers follow
 };
 
 template <int D>
@@ -67,9 +69,21 @@ struct Cfg {
     static constexpr int kNumBars = kBarSlotEmpty + kStages;
     static constexpr int kBarOff = (2 + kStages) * kTileBytes;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + alignment slack
-    // TMEM columns of S_t (P_t aliases its first 64) and O_t.
+    // TMEM columns.  At D = 64 everything fits apart: S0 S1 (128 each), P0 P1 (64 each),
+    // O0 O1 (64 each) = 512, so the next Q K^T can overwrite S while P is still being
+    // computed.  At D = 128, P_t is written over the first 64 columns of S_t.
+    static constexpr bool kSepP = (D == 64);
+    // Pairs (of 16 per 32-column chunk) whose 2^x runs on the FMA pipe in full tiles,
+    // to take load off the MUFU unit; worth it only when a score_mod already spends MUFU
+    // time (tanh), per measurement.
+    static constexpr int emu_pairs(int score) { return score != 0 ? 4 : 0; }
     __device__ static constexpr uint32_t colS(int t) { return (uint32_t)t * 128u; }
-    __device__ static constexpr uint32_t colO(int t) { return 256u + (uint32_t)t * (uint32_t)D; }
+    __device__ static constexpr uint32_t colP(int t) {
+        return kSepP ? 256u + (uint32_t)t * 64u : (uint32_t)t * 128u;
+    }
+    __device__ static constexpr uint32_t colO(int t) {
+        return kSepP ? 384u + (uint32_t)t * 64u : 256u + (uint32_t)t * (uint32_t)D;
+    }
 };
 
 struct Unit {
@@ -164,14 +178,13 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
     __syncwarp();
     uint32_t kv_pos = 0, q_iter = 0;
     bool ok = true;
-    int tn = 0;
-    (void)tn;
+    FA_TRACE_DECL
     for (int k = 0; ok; ++k) {
         const int u = unit_of_round(k);
         if (u >= p.n_units) break;
         const Unit un = decode_unit(p, u);
         if (un.E == 0) continue;
-        FA_TRACE_EV(0, tn, 40);
+        FA_TRACE_EV(0, 40);
         if (!wait(kBarQEmpty, (q_iter & 1u) ^ 1u)) { ok = false; break; }
         const int q0 = 2 * un.pair;
         const int nq = (q0 + 1 < p.QB) ? 2 : 1;
@@ -188,9 +201,9 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
             for (int which = 0; which < 2; ++which) {
                 const int s = (int)(kv_pos % C::kStages);
                 const uint32_t ph = (kv_pos / C::kStages) & 1u;
-                FA_TRACE_EV(0, tn, 30 + which);
+                FA_TRACE_EV(0, 30 + which);
                 if (!wait(C::kBarSlotEmpty + s, ph ^ 1u)) { ok = false; break; }
-                FA_TRACE_EV(0, tn, 32 + which);
+                FA_TRACE_EV(0, 32 + which);
                 mbar_arrive_expect_tx_if(leader, bar(kBarSlotFull + s), (uint32_t)C::kTileBytes);
                 const CUtensorMap* tm = which ? tmv : tmk;
                 for (int c = 0; c < C::kChunks; ++c)
@@ -245,7 +258,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
     // two 8-row atoms (SBO = 1024 bytes), 64-column boxes 16 KB apart (LBO).
     auto issue_pv = [&](int t, int slot, bool accumulate) {
         const uint32_t d = tmem + C::colO(t);
-        const uint32_t pa = tmem + C::colS(t);
+        const uint32_t pa = tmem + C::colP(t);
         const uint64_t vd = make_sdesc_sw128(sKV + slot * C::kTileBytes, 16384, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBlock / 16; ++kk) {
@@ -255,10 +268,21 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
     };
 
     uint32_t kv_pos = 0, q_iter = 0;
-    uint32_t pf_cnt[2] = {0u, 0u}, of_cnt[2] = {0u, 0u};
+    uint32_t pf_cnt[2] = {0u, 0u}, of_cnt[2] = {0u, 0u}, qk_cnt[2] = {0u, 0u};
     bool ok = true;
-    int tn = 0;
-    (void)tn;
+    FA_TRACE_DECL
+    // S_t = Q_t K^T into TMEM; with separate P it first waits until the softmax holds the
+    // previous S_t in registers.
+    auto do_qk = [&](int t, int slot) -> bool {
+        if constexpr (C::kSepP) {
+            if (!wait(kBarSFree + t, (qk_cnt[t] & 1u) ^ 1u)) return false;
+            tc_fence_after();
+        }
+        ++qk_cnt[t];
+        issue_qk(t, slot);
+        tc_commit_if(leader, bar(kBarSFull + t));
+        return true;
+    };
     for (int k = 0; ok; ++k) {
         const int u = unit_of_round(k);
         if (u >= p.n_units) break;
@@ -272,6 +296,20 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
         const uint32_t kbase = kv_pos;
         kv_pos += 2u * (uint32_t)un.E;
         int ndone[2] = {0, 0};
+        // O_t += P_t V once the softmax has published P_t.
+        auto do_pv = [&](int t, int slot) -> bool {
+            FA_TRACE_EV(1, 16 + t);
+            if (!wait(kBarPFull + t, pf_cnt[t] & 1u)) return false;
+            FA_TRACE_EV(1, 18 + t);
+            ++pf_cnt[t];
+            if (ndone[t] == 0 && !wait(kBarOFree + t, (of_cnt[t] & 1u) ^ 1u)) return false;
+            tc_fence_after();
+            issue_pv(t, slot, ndone[t] > 0);
+            if constexpr (C::kSepP) tc_commit_if(leader, bar(kBarPVDone + t));
+            if (ndone[t] + 1 == nl[t]) tc_commit_if(leader, bar(kBarOFull + t));
+            ++ndone[t];
+            return true;
+        };
         EntryReader er;
         er.init(un.entries, un.E);
         int code = er.get(0);
@@ -280,11 +318,9 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
             const int s = (int)(pos % C::kStages);
             if (!wait(kBarSlotFull + s, (pos / C::kStages) & 1u)) { ok = false; break; }
             tc_fence_after();
-            for (int t = 0; t < 2; ++t)
-                if (code & (t ? kLive1 : kLive0)) {
-                    issue_qk(t, s);
-                    tc_commit_if(leader, bar(kBarSFull + t));
-                }
+            for (int t = 0; t < 2 && ok; ++t)
+                if (code & (t ? kLive1 : kLive0)) ok = do_qk(t, s);
+            if (!ok) break;
             tc_commit_if(leader, bar(C::kBarSlotEmpty + s));
             if (un.E == 1) tc_commit_if(leader, bar(kBarQEmpty));
         }
@@ -293,29 +329,25 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
             const int next = has_next ? er.get(e + 1) : 0;
             const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u, kpos = vpos + 1u;
             const int vs = (int)(vpos % C::kStages), ks = (int)(kpos % C::kStages);
-            FA_TRACE_EV(1, tn, 22);
+            FA_TRACE_EV(1, 22);
             if (!wait(kBarSlotFull + vs, (vpos / C::kStages) & 1u)) { ok = false; break; }
             if (has_next && !wait(kBarSlotFull + ks, (kpos / C::kStages) & 1u)) { ok = false; break; }
-            FA_TRACE_EV(1, tn, 23);
+            FA_TRACE_EV(1, 23);
             tc_fence_after();
-            for (int t = 0; t < 2; ++t) {
-                if (code & (t ? kLive1 : kLive0)) {
-                    FA_TRACE_EV(1, tn, 16 + t);
-                    if (!wait(kBarPFull + t, pf_cnt[t] & 1u)) { ok = false; break; }
-                    FA_TRACE_EV(1, tn, 18 + t);
-                    ++pf_cnt[t];
-                    if (ndone[t] == 0 && !wait(kBarOFree + t, (of_cnt[t] & 1u) ^ 1u)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    issue_pv(t, vs, ndone[t] > 0);
-                    if (ndone[t] + 1 == nl[t]) tc_commit_if(leader, bar(kBarOFull + t));
-                    ++ndone[t];
+            if constexpr (C::kSepP) {
+                // Per tile: the next S first (it only needs the softmax to have read the
+                // current S), then P.V of the current entry.  Tile 0 runs ahead of tile 1
+                // (the softmax groups take turns), so tile 0 is served first.
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (next & (t ? kLive1 : kLive0)) ok = do_qk(t, ks);
+                    if (ok && (code & (t ? kLive1 : kLive0))) ok = do_pv(t, vs);
                 }
-                if (next & (t ? kLive1 : kLive0)) {
-                    issue_qk(t, ks);
-                    tc_commit_if(leader, bar(kBarSFull + t));
+            } else {
+                // P_t lives in S_t: P.V of the current entry must be issued before the
+                // next Q K^T overwrites it.
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (code & (t ? kLive1 : kLive0)) ok = do_pv(t, vs);
+                    if (ok && (next & (t ? kLive1 : kLive0))) ok = do_qk(t, ks);
                 }
             }
             if (!ok) break;
@@ -339,6 +371,40 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
 
 // ------------------------------------------------------------------ softmax (warps 4-11)
 
+// P = 2^(x - base) for one 128-wide row, packed to 16-bit pairs and stored to TMEM at tP
+// in four 32-column chunks; returns the (two-lane) row sum.  EMU of every 16 pairs use
+// the FMA-pipe exp2 (only for tiles without masked positions), the rest MUFU ex2.
+template <bool BF16, bool SCORE, int EMU>
+__device__ __forceinline__ float2 softmax_p_row(const float2 (&x)[64], float2 nb2, float2 k2,
+                                                uint32_t tP) {
+    float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                    make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int chunk = 0; chunk < 4; ++chunk) {
+        // All exponentials of the chunk first (independent, so their latencies overlap),
+        // then the sums and the 16-bit packing.
+        float2 pe[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float2 a = SCORE ? __fadd2_rn(x[chunk * 16 + i], nb2)
+                                   : __ffma2_rn(x[chunk * 16 + i], k2, nb2);
+            if ((i * EMU) % 16 < EMU) {
+                pe[i] = exp2_fma2(a);
+            } else {
+                pe[i] = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+            }
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            rs[i & 3] = __fadd2_rn(rs[i & 3], pe[i]);
+            pk[i] = pack2<BF16>(pe[i].x, pe[i].y);
+        }
+        tmem_st_32x32b_x16(tP + chunk * 16, pk);
+    }
+    return __fadd2_rn(__fadd2_rn(rs[0], rs[1]), __fadd2_rn(rs[2], rs[3]));
+}
+
 template <int D, bool BF16>
 __device__ __forceinline__ void store_row_zero(const FwdParams& p, const Unit& un, int q) {
     uint16_t* o = reinterpret_cast<uint16_t*>(p.out) + un.b * p.out_stride[0] +
@@ -348,7 +414,7 @@ __device__ __forceinline__ void store_row_zero(const FwdParams& p, const Unit& u
     if (p.lse) p.lse[((int64_t)un.b * p.H + un.h) * p.Q_LEN + q] = -INFINITY;
 }
 
-template <int D, bool BF16, bool SCORE>
+template <int D, bool BF16, int SCORE>
 __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t tmem,
                              volatile int* abort_flag) {
     using C = Cfg<D>;
@@ -357,6 +423,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
     const int row = wq * 32 + lane;
     const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_bits + C::colS(t);
+    const uint32_t tP = tmem + lane_bits + C::colP(t);
     const uint32_t tO = tmem + lane_bits + C::colO(t);
     const int live_bit = t ? kLive1 : kLive0;
     const int full_bit = t ? kFull1 : kFull0;
@@ -364,30 +431,29 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
     auto wait = [&](int i, uint32_t par) {
         return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
     };
-    const bool has_softcap = SCORE && (p.score_kind & FA_SCORE_SOFTCAP);
-    const bool has_alibi = SCORE && (p.score_kind & FA_SCORE_ALIBI);
+    constexpr bool has_softcap = (SCORE & FA_SCORE_SOFTCAP) != 0;
+    constexpr bool has_alibi = (SCORE & FA_SCORE_ALIBI) != 0;
 
-    uint32_t sf_cnt = 0, of_cnt = 0;
+    uint32_t sf_cnt = 0, of_cnt = 0, pst_cnt = 0;
     const int tslot = 2 + (int)(threadIdx.x >> 5) - 4;  // one trace slot per softmax warp
-    int tn = 0;
+    FA_TRACE_DECL
     (void)tslot;
-    (void)tn;
     for (int k = 0;; ++k) {
         const int u = unit_of_round(k);
         if (u >= p.n_units) break;
         const Unit un = decode_unit(p, u);
         const int qblk = 2 * un.pair + t;
-        if (qblk >= p.QB) continue;
-        const int q = qblk * kBlock + row;
         int nl0 = 0, nl1 = 0;
         if (un.E > 0) count_live(un.entries, un.E, nl0, nl1);
         const int nl = t ? nl1 : nl0;
+        if (qblk >= p.QB) continue;
         if (nl == 0) {
-            store_row_zero<D, BF16>(p, un, q);
+            store_row_zero<D, BF16>(p, un, qblk * kBlock + row);
             continue;
         }
+        const int q = qblk * kBlock + row;
         float slope_log2 = 0.f;
-        if (has_alibi) {
+        if constexpr (has_alibi) {
             float slope;
             if (p.alibi_slopes) {
                 slope = __ldg(p.alibi_slopes + un.h);
@@ -409,9 +475,9 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             if (!(code & live_bit)) continue;
             const int j = code & 0xFFFF;
             const bool full = (code & full_bit) != 0;
-            FA_TRACE_EV(tslot, tn, 1);
+            FA_TRACE_EV(tslot, 1);
             if (!wait(kBarSFull + t, sf_cnt & 1u)) { ok = false; break; }
-            FA_TRACE_EV(tslot, tn, 2);
+            FA_TRACE_EV(tslot, 2);
             ++sf_cnt;
             tc_fence_after();
             // S row of this thread: 128 fp32 scores held as 64 pairs.
@@ -428,9 +494,14 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                     x[i] = make_float2(__uint_as_float(sr[i >> 4][(2 * i) & 31]),
                                        __uint_as_float(sr[i >> 4][(2 * i + 1) & 31]));
             }
-            FA_TRACE_EV(tslot, tn, 3);
+            if constexpr (C::kSepP) {
+                // S is in registers: the next Q K^T may overwrite it.
+                tc_fence_before();
+                mbar_arrive_warp(bar(kBarSFree + t));
+            }
+            FA_TRACE_EV(tslot, 3);
             const int kv0 = j * kBlock;
-            if constexpr (SCORE) {
+            if constexpr (SCORE != 0) {
                 // score_mod on every position of the tile, in log2 units; masked
                 // positions are set to -inf afterwards (the mask decides liveness).
                 const float2 inv2 = make_float2(p.inv_softcap_scale, p.inv_softcap_scale);
@@ -442,13 +513,13 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
 #pragma unroll
                 for (int i = 0; i < 64; ++i) {
                     float2 y;
-                    if (has_softcap) {
+                    if constexpr (has_softcap) {
                         const float2 a = __fmul2_rn(x[i], inv2);
                         y = __fmul2_rn(cap2, make_float2(tanh_approx(a.x), tanh_approx(a.y)));
                     } else {
                         y = __fmul2_rn(x[i], sc2);
                     }
-                    if (has_alibi) {
+                    if constexpr (has_alibi) {
                         y = __ffma2_rn(sl2, pos, y);
                         pos = __fadd2_rn(pos, two);
                     }
@@ -479,18 +550,20 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                     }
                 }
             }
-            // Row max with three-input max: four independent chains over quarters.
-            float mc[4];
+            // Row max with three-input max: eight independent chains over eighths.
+            float mc[8];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) mc[c] = fmaxf(x[16 * c].x, x[16 * c].y);
+            for (int c = 0; c < 8; ++c) mc[c] = fmaxf(x[8 * c].x, x[8 * c].y);
 #pragma unroll
-            for (int i = 1; i < 16; ++i)
+            for (int i = 1; i < 8; ++i)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) mc[c] = max3(mc[c], x[16 * c + i].x, x[16 * c + i].y);
+                for (int c = 0; c < 8; ++c) mc[c] = max3(mc[c], x[8 * c + i].x, x[8 * c + i].y);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) mc[c] = fmaxf(mc[c], mc[c + 4]);
             float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
-            if constexpr (!SCORE) mt *= p.scale_log2;
+            if constexpr (SCORE == 0) mt *= p.scale_log2;
             const float m_new = fmaxf(m, mt);
-            FA_TRACE_EV(tslot, tn, 4);
+            FA_TRACE_EV(tslot, 4);
             const bool need = m_new > m + kRescaleThreshold;
             const bool any_need = __any_sync(kFullMask, need);
             float alpha = 1.0f;
@@ -499,25 +572,21 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                 m = m_new;
             }
             const float base = (m == -INFINITY) ? 0.f : m;
-            // P = 2^(x - base) in 16-bit pairs, written over S in four chunks.
-            float2 rs = make_float2(0.f, 0.f);
+            FA_TRACE_EV(tslot, 9);
+            if constexpr (C::kSepP) {
+                // The previous P.V of this tile must be done before P and O are touched.
+                if (!wait(kBarPVDone + t, (pst_cnt & 1u) ^ 1u)) { ok = false; break; }
+                tc_fence_after();
+            }
+            FA_TRACE_EV(tslot, 10);
+            ++pst_cnt;
+            // P = 2^(x - base) in 16-bit pairs, written to TMEM in four chunks.
             const float2 nb2 = make_float2(-base, -base);
             const float2 k2 = make_float2(p.scale_log2, p.scale_log2);
-#pragma unroll
-            for (int chunk = 0; chunk < 4; ++chunk) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float2 a = SCORE ? __fadd2_rn(x[chunk * 16 + i], nb2)
-                                           : __ffma2_rn(x[chunk * 16 + i], k2, nb2);
-                    const float2 pe = make_float2(ex2_approx(a.x), ex2_approx(a.y));
-                    rs = __fadd2_rn(rs, pe);
-                    pk[i] = pack2<BF16>(pe.x, pe.y);
-                }
-                tmem_st_32x32b_x16(tS + chunk * 16, pk);
-            }
+            const float2 rs = full ? softmax_p_row<BF16, (SCORE != 0), C::emu_pairs(SCORE)>(x, nb2, k2, tP)
+                                   : softmax_p_row<BF16, (SCORE != 0), 0>(x, nb2, k2, tP);
             l = fmaf(l, alpha, rs.x + rs.y);
-            FA_TRACE_EV(tslot, tn, 5);
+            FA_TRACE_EV(tslot, 5);
             if (any_need && done > 0) {
                 // Rescale O only now, after S has left the registers.
                 const float2 al2 = make_float2(alpha, alpha);
@@ -539,13 +608,13 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(bar(kBarPFull + t));
-            FA_TRACE_EV(tslot, tn, 6);
+            mbar_arrive_warp(bar(kBarPFull + t));
+            FA_TRACE_EV(tslot, 6);
             ++done;
         }
         if (!ok) return;
         // Epilogue: O / l in the output dtype, and the natural-log lse.
-        FA_TRACE_EV(tslot, tn, 7);
+        FA_TRACE_EV(tslot, 7);
         if (!wait(kBarOFull + t, of_cnt & 1u)) return;
         ++of_cnt;
         tc_fence_after();
@@ -571,14 +640,14 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             p.lse[((int64_t)un.b * p.H + un.h) * p.Q_LEN + q] =
                 (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
         tc_fence_before();
-        mbar_arrive(bar(kBarOFree + t));
-        FA_TRACE_EV(tslot, tn, 8);
+        mbar_arrive_warp(bar(kBarOFree + t));
+        FA_TRACE_EV(tslot, 8);
     }
 }
 
 // ------------------------------------------------------------------ kernel
 
-template <int D, bool BF16, bool SCORE>
+template <int D, bool BF16, int SCORE>
 __global__ void __launch_bounds__(kThreadsFwd, 1)
 attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tmq,
                 const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
@@ -597,9 +666,11 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
         mbar_init(bars + 8u * kBarQEmpty, 1);
         for (int t = 0; t < 2; ++t) {
             mbar_init(bars + 8u * (kBarSFull + t), 1);
-            mbar_init(bars + 8u * (kBarPFull + t), 128);
+            mbar_init(bars + 8u * (kBarPFull + t), 4);   // one arrival per softmax warp
             mbar_init(bars + 8u * (kBarOFull + t), 1);
-            mbar_init(bars + 8u * (kBarOFree + t), 128);
+            mbar_init(bars + 8u * (kBarOFree + t), 4);
+            mbar_init(bars + 8u * (kBarSFree + t), 4);
+            mbar_init(bars + 8u * (kBarPVDone + t), 1);
         }
         mbar_init(bars + 8u * kBarDrain, 1);
         for (int s = 0; s < C::kStages; ++s) {
@@ -638,7 +709,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
     if (warp == 2) tmem_dealloc(tmem, 512);
 }
 
-template <int D, bool BF16, bool SCORE>
+template <int D, bool BF16, int SCORE>
 cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                      const CUtensorMap& tv, int grid, cudaStream_t stream) {
     auto kern = attn_fwd_kernel<D, BF16, SCORE>;
@@ -651,20 +722,18 @@ cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMa
 
 }  // namespace
 
-cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, bool has_score,
+cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, int score_kind,
                             const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             int grid, cudaStream_t stream) {
 #define FA_CASE(DD, BB, SS)                                                 \
-    if (D == DD && bf16 == BB && has_score == SS)                           \
+    if (D == DD && bf16 == BB && score_kind == SS)                          \
         return launch_t<DD, BB, SS>(p, tq, tk, tv, grid, stream);
-    FA_CASE(64, true, false)
-    FA_CASE(64, true, true)
-    FA_CASE(64, false, false)
-    FA_CASE(64, false, true)
-    FA_CASE(128, true, false)
-    FA_CASE(128, true, true)
-    FA_CASE(128, false, false)
-    FA_CASE(128, false, true)
+#define FA_CASES(DD, BB) FA_CASE(DD, BB, 0) FA_CASE(DD, BB, 1) FA_CASE(DD, BB, 2) FA_CASE(DD, BB, 3)
+    FA_CASES(64, true)
+    FA_CASES(64, false)
+    FA_CASES(128, true)
+    FA_CASES(128, false)
+#undef FA_CASES
 #undef FA_CASE
     return cudaErrorInvalidValue;
 }

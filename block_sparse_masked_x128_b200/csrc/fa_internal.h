@@ -71,7 +71,7 @@ cudaError_t launch_mask_lists(const MaskSpec& spec, int separate_full, int maskB
 fa_status_t record_error(fa_status_t status, const char* message);
 fa_status_t record_ok();
 
-cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, bool has_score,
+cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, int score_kind,
                             const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             int grid, cudaStream_t stream);
 

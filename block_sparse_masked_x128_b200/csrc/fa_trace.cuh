@@ -16,14 +16,18 @@ constexpr int kTraceCap = 16384;
 #ifdef FA_TRACE
 // Defined in the one translation unit that includes this header (attn_fwd.cu).
 static __device__ unsigned long long* g_fa_trace = nullptr;
-__device__ __forceinline__ void fa_trace_event(int slot, int& n, int tag) {
-    if (blockIdx.x == 0 && (threadIdx.x & 31) == 0 && g_fa_trace && n < fa::kTraceCap) {
-        g_fa_trace[slot * fa::kTraceCap + n] =
-            ((unsigned long long)tag << 56) | (clock64() & 0x00FFFFFFFFFFFFFFull);
-    }
-    ++n;
-}
-#define FA_TRACE_EV(slot, n, tag) fa_trace_event((slot), (n), (tag))
+// Declares the role's trace cursor; the buffer pointer is read once, kept in a register.
+#define FA_TRACE_DECL                                                                \
+    unsigned long long* fa_tbuf_ = (blockIdx.x == 0) ? g_fa_trace : nullptr;         \
+    int fa_tn_ = 0;
+#define FA_TRACE_EV(slot, tag)                                                       \
+    do {                                                                             \
+        if (fa_tbuf_ && (threadIdx.x & 31) == 0 && fa_tn_ < fa::kTraceCap)           \
+            fa_tbuf_[(slot) * fa::kTraceCap + fa_tn_] =                              \
+                ((unsigned long long)(tag) << 56) | (clock64() & 0x00FFFFFFFFFFFFFFull); \
+        ++fa_tn_;                                                                    \
+    } while (0)
 #else
-#define FA_TRACE_EV(slot, n, tag) ((void)0)
+#define FA_TRACE_DECL
+#define FA_TRACE_EV(slot, tag) ((void)0)
 #endif

@@ -38,6 +38,13 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// One arrival per warp: every lane has done its own work and fences before calling; the
+// warp synchronises and lane 0 arrives (barriers expecting one arrival per warp).
+__device__ __forceinline__ void mbar_arrive_warp(uint32_t bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
@@ -48,6 +55,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -297,6 +317,31 @@ __device__ __forceinline__ float tanh_approx(float x) {
     float y;
     asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^a for two values on the FMA pipe (no MUFU), for a <= 127.  Method: Cody-Waite
+// reduction a = n + f with n = round(a) (obtained by adding 1.5 * 2^23, which leaves n in
+// the low mantissa bits) and |f| <= 1/2; 2^f by a degree-3 polynomial fitted here for
+// minimal relative error on [-1/2, 1/2] (Lawson-weighted least squares, max relative error
+// 7.5e-5); 2^n by adding n to the exponent field.  Inputs below -126 are clamped to -126,
+// so the result is never below about 2^-127 (callers that need exact zeros must not use it).
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716648042202f;
+__device__ __forceinline__ float2 exp2_fma2(float2 a) {
+    const float2 rnd = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+    a = make_float2(fmaxf(a.x, -126.0f), fmaxf(a.y, -126.0f));
+    const float2 t = __fadd2_rn(a, rnd);                                   // rnd + n
+    const float2 neg_n = __ffma2_rn(t, make_float2(-1.0f, -1.0f), rnd);    // -n, exact
+    const float2 f = __fadd2_rn(a, neg_n);                                 // a - n, exact
+    float2 q = __ffma2_rn(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
+    q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
+    q = __ffma2_rn(q, f, make_float2(kExp2C0, kExp2C0));
+    // bits(t) = bits(rnd) + n and bits(rnd) has nine low zero bits, so (bits(t) << 23) is
+    // n in the exponent field.
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // Pack two floats into one 32-bit register of two 16-bit values, `lo` in bits 0-15.

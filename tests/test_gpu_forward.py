@@ -105,13 +105,20 @@ def test_packed_documents_equal_separate_runs():
 
 @pytest.mark.parametrize("kind,window", [(C, 0), (C | SW, 300), (C | DOC, 0)])
 def test_separate_full_blocks_does_not_change_the_result(kind, window):
+    # Without separate full blocks every live tile is masked like a partial one (and takes
+    # the MUFU exp2 path), so the two results agree to rounding, each within tolerance.
     fa = fa_module()
     doc = wl.doc_ids_from_lengths([700, 900, 448]) if kind & DOC else None
-    g = torch.Generator().manual_seed(6)
-    q, k, v = (torch.randn(1, 2, 2048, 64, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
-    a = fa.flex_attention(q, k, v, gpu_block_mask(kind, None, None, 2048, 2048, window, doc, True))
-    b = fa.flex_attention(q, k, v, gpu_block_mask(kind, None, None, 2048, 2048, window, doc, False))
-    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    w = wl.Workload("separate_full", B=1, H=2, S=2048, D=64, dtype="bf16", mask_kind=kind,
+                    window=window, seed=6)
+    q, k, v = wl.make_qkv(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    a = fa.flex_attention(qd, kd, vd, gpu_block_mask(kind, None, None, 2048, 2048, window, doc, True))
+    b = fa.flex_attention(qd, kd, vd, gpu_block_mask(kind, None, None, 2048, 2048, window, doc, False))
+    O, L = run_oracle(w, q, k, v, doc)
+    compare(a[0], a[1], O, L)
+    compare(b[0], b[1], O, L)
+    assert (a[0].float() - b[0].float()).abs().max().item() < 1e-2
 
 
 def test_strided_layout_equals_contiguous():
