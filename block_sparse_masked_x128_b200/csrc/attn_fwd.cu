@@ -41,6 +41,14 @@ namespace fa {
 namespace {
 
 constexpr int kThreadsFwd = 384;
+// Register budgets (setmaxnreg): the launch gives every thread 65536 / 384 rounded down to a
+// multiple of 8 = 168; the TMA/MMA warpgroup drops to 80 and the two softmax warpgroups rise
+// to 208, within the launched pool.
+constexpr int kRegsAtLaunch = 168;
+constexpr int kRegsProducer = 80;
+constexpr int kRegsSoftmax = 208;
+static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreadsFwd * kRegsAtLaunch,
+              "register split exceeds the launched pool");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -690,17 +698,16 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
     const uint32_t tmem = *tmem_slot;
 
     // Registers: the TMA/MMA warpgroup needs few, the softmax warpgroups hold a 128-wide
-    // score row each.  4 warps x 80 + 8 warps x 208 fits the 384 x 168 launched.  Each
-    // role runs inside the branch of its own budget.
+    // score row each (budgets above).  Each role runs inside the branch of its own budget.
     if (warp < 4) {
-        regs_dec<80>();
+        regs_dec<kRegsProducer>();
         if (warp == 0) {
             producer_role<D>(p, &tmq, &tmk, &tmv, sbase, bars, abort_flag);
         } else if (warp == 1) {
             mma_role<D, BF16>(p, sbase, bars, tmem, abort_flag);
         }
     } else {
-        regs_inc<208>();
+        regs_inc<kRegsSoftmax>();
         softmax_role<D, BF16, SCORE>(p, (warp - 4) >> 2, bars, tmem, abort_flag);
     }
     tc_fence_before();
@@ -713,8 +720,13 @@ template <int D, bool BF16, int SCORE>
 cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                      const CUtensorMap& tv, int grid, cudaStream_t stream) {
     auto kern = attn_fwd_kernel<D, BF16, SCORE>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg<D>::kSmemBytes);
+    // setmaxnreg.inc waits for registers from the launched pool; refuse to launch a build
+    // whose per-thread register count would make that pool smaller than the split needs.
+    cudaFuncAttributes attr;
+    cudaError_t e = cudaFuncGetAttributes(&attr, kern);
+    if (e != cudaSuccess) return e;
+    if (attr.numRegs < kRegsAtLaunch) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemBytes);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreadsFwd, Cfg<D>::kSmemBytes, stream>>>(p, tq, tk, tv);
     return cudaGetLastError();

@@ -9,7 +9,7 @@
 #include <cstdint>
 
 namespace fa {
-constexpr int kTraceSlots = 16;
+constexpr int kTraceSlots = 20;
 constexpr int kTraceCap = 16384;
 }  // namespace fa
 

@@ -14,9 +14,9 @@
 //      tiles are evaluated element by element by the whole CTA.  Live tiles are then
 //      compacted into ascending lists with warp ballots and popc prefix sums.
 //   2. schedule_kernel: one CTA per work unit (a pair of adjacent query blocks) merges
-//      the two tiles' partial and full lists into one ascending list of kv blocks with
-//      per-tile live/full flags, so the forward kernel loads each K/V tile once for both
-//      query tiles.  The unit's cost is the number of live tiles it holds.
+//      the two tiles' partial and full lists into one list of kv blocks, nearest first
+//      (descending), with per-tile live/full flags, so the forward kernel loads each K/V
+//      tile once for both query tiles.  The unit's cost is the number of live tiles.
 //   3. lpt_order_kernel: ranks the units of each stored (b, h) by descending cost (ties
 //      by index) so the persistent forward kernel hands the longest units out first.
 #include <climits>
@@ -210,10 +210,13 @@ schedule_kernel(int QB, int KVB, int NP, const int32_t* __restrict__ kv_num,
     }
     const size_t unit = (size_t)bh * NP + p;
     int32_t* out = sched_entries + unit * KVB;
+    // Entries go out nearest first (descending kv block): the diagonal tiles come first, so
+    // a row's running max is usually settled by its first tile (with ALiBi the bias grows
+    // toward the diagonal, and ascending order would raise the max on every tile).
     int cnt = 0, l0 = 0, l1 = 0;
     for (int jb = 0; jb < KVB; jb += kThreads) {
-        const int j = jb + tid;
-        const int c = (j < KVB) ? s_code[j] : 0;
+        const int j = KVB - 1 - (jb + tid);
+        const int c = (j >= 0) ? s_code[j] : 0;
         const unsigned b = __ballot_sync(0xffffffffu, c != 0);
         const unsigned b0 = __ballot_sync(0xffffffffu, (c & (kLive0 >> 16)) != 0);
         const unsigned b1 = __ballot_sync(0xffffffffu, (c & (kLive1 >> 16)) != 0);
