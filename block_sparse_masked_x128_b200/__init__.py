@@ -42,7 +42,7 @@ FA_DTYPE_BF16 = 1
 
 EXPORTED = ("fa_create_block_mask", "fa_forward", "fa_block_mask_get", "fa_get_device_status",
             "fa_destroy_block_mask", "fa_status_string", "fa_last_error_message",
-            "fa_create_block_mask_noalloc")
+            "fa_create_block_mask_noalloc", "fa_debug_set_stall")
 
 
 class FaMaskParams(ctypes.Structure):
@@ -94,6 +94,8 @@ _lib.fa_status_string.argtypes = [ctypes.c_int]
 _lib.fa_status_string.restype = ctypes.c_char_p
 _lib.fa_last_error_message.argtypes = []
 _lib.fa_last_error_message.restype = ctypes.c_char_p
+_lib.fa_debug_set_stall.argtypes = [ctypes.c_int32]
+_lib.fa_debug_set_stall.restype = _status
 
 
 class FaError(RuntimeError):
@@ -191,6 +193,11 @@ def fa_get_device_status(block_mask: int, stream=None) -> int:
 
 def fa_destroy_block_mask(block_mask: int) -> None:
     _lib.fa_destroy_block_mask(block_mask)
+
+
+def fa_debug_set_stall(enable: bool) -> None:
+    """Test hook: make every later forward's bounded K wait run out (see the C header)."""
+    _check(_lib.fa_debug_set_stall(1 if enable else 0), "fa_debug_set_stall")
 
 
 # ---------------------------------------------------------------- convenience API

@@ -37,6 +37,17 @@ extern "C" int fa_debug_set_trace_buffer(void* device_ptr) {
 }
 #endif
 
+// Test hook for failure detection: while nonzero, every forward's producer warp stops after
+// the first unit's Q load, so the MMA warp's bounded wait for K runs out, the kernel unwinds
+// and the mask's status word reports the timeout.  Nothing faults, traps or hangs.
+static __device__ int g_fa_stall_loads = 0;
+
+extern "C" fa_status_t fa_debug_set_stall(int32_t enable) {
+    const int v = enable ? 1 : 0;
+    const cudaError_t e = cudaMemcpyToSymbol(g_fa_stall_loads, &v, sizeof(v));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 namespace fa {
 namespace {
 
@@ -186,6 +197,7 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
     __syncwarp();
     uint32_t kv_pos = 0, q_iter = 0;
     bool ok = true;
+    const bool stall = *reinterpret_cast<volatile int*>(&g_fa_stall_loads) != 0;
     FA_TRACE_DECL
     for (int k = 0; ok; ++k) {
         const int u = unit_of_round(k);
@@ -202,6 +214,10 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
                 tma_load_4d_if(leader, sQ + t * C::kTileBytes + c * 16384, tmq, bar(kBarQFull),
                                c * 64, (q0 + t) * kBlock, un.h, un.b);
         ++q_iter;
+        if (stall) {  // test hook: let Q land, then never load K or V
+            drain_wait(bar(kBarQFull), (q_iter - 1) & 1u);
+            return;
+        }
         EntryReader er;
         er.init(un.entries, un.E);
         for (int e = 0; e < un.E && ok; ++e) {
