@@ -196,7 +196,7 @@ def oracle_sample_rate(w: wl.Workload, q, k, v, doc, budget_s: float, rows_per_c
     qn, kn, vn = (t.float().numpy() for t in (q, k, v))
     live_row = _live_per_row(w, doc)
     rows_done, live, t_total = 0, 0, 0.0
-    while t_total < budget_s:
+    while rows_done == 0 or t_total < budget_s:   # at least one chunk
         b = int(rng.integers(0, w.B))
         h = int(rng.integers(0, w.H))
         rows = np.sort(rng.choice(w.S, size=min(rows_per_chunk, w.S), replace=False))
@@ -391,7 +391,7 @@ def run_reference(args, w: wl.Workload, world: int, rank: int) -> dict:
     t0 = time.perf_counter()
     tot_live, tot_t, tot_rows = 0, 0.0, 0
     for i in range(args.steps):
-        r = oracle_sample_rate(w, q, k, v, doc, 0.0, rows_per_chunk=rows, seed=i)
+        r = oracle_sample_rate(w, q, k, v, doc, per_step, rows_per_chunk=rows, seed=i)
         tot_live += r["live_positions"]
         tot_t += r["seconds"]
         tot_rows += r["rows"]

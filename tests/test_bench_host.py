@@ -103,3 +103,21 @@ def test_config_names_the_workload():
     assert c["workload"] == wl.WORKLOADS[4].name and c["parallelism"] == "dp2"
     assert "softcap" in c["score_mod"] and "alibi" in c["score_mod"]
     assert c["global_batch"] == 2
+
+
+def test_reference_arm_times_bounded_oracle_samples():
+    import argparse
+    args = argparse.Namespace(steps=2, warmup=3, reference_budget_s=0.5)
+    w = wl.WORKLOADS[1].scaled(S=1024)
+    r = bench.run_reference(args, w, 1, 0)
+    assert r["impl"] == "reference" and r["value"] > 0 and r["dtype"] == "f64"
+    assert r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["value"] == r["value"]
+    assert r["e2e"]["value"] == r["value"] and r["e2e"]["h2d_bytes_per_step"] == 0
+    assert r["steps"] == 2 and r["warmup"] == 3
+
+
+def test_oracle_sample_rate_runs_at_least_one_chunk():
+    w = wl.WORKLOADS[0]
+    q, k, v = wl.make_qkv(w)
+    r = bench.oracle_sample_rate(w, q, k, v, None, 0.0, rows_per_chunk=8)
+    assert r["rows"] == 8 and r["value"] > 0
