@@ -384,7 +384,7 @@ def run_reference(args, w: wl.Workload, world: int, rank: int) -> dict:
     q, k, v = wl.make_qkv(w)
     doc = wl.make_doc_ids(w)
     per_step = max(0.02, args.reference_budget_s / max(1, args.steps + args.warmup))
-    rows = 16
+    rows = 256
     oracle_sample_rate(w, q, k, v, doc, 0.0, rows_per_chunk=rows)  # warm the imports
     for _ in range(args.warmup):
         oracle_sample_rate(w, q, k, v, doc, 0.0, rows_per_chunk=rows)

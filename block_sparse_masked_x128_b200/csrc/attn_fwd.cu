@@ -53,11 +53,11 @@ namespace {
 
 constexpr int kThreadsFwd = 384;
 // Register budgets (setmaxnreg): the launch gives every thread 65536 / 384 rounded down to a
-// multiple of 8 = 168; the TMA/MMA warpgroup drops to 80 and the two softmax warpgroups rise
-// to 208, within the launched pool.
+// multiple of 8 = 168; the TMA/MMA warpgroup drops to 104 (at 80 its issue loops spill) and
+// the two softmax warpgroups rise to 200: exactly the launched pool.
 constexpr int kRegsAtLaunch = 168;
-constexpr int kRegsProducer = 80;
-constexpr int kRegsSoftmax = 208;
+constexpr int kRegsProducer = 104;
+constexpr int kRegsSoftmax = 200;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreadsFwd * kRegsAtLaunch,
               "register split exceeds the launched pool");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
@@ -342,8 +342,9 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
             const int s = (int)(pos % C::kStages);
             if (!wait(kBarSlotFull + s, (pos / C::kStages) & 1u)) { ok = false; break; }
             tc_fence_after();
-            for (int t = 0; t < 2 && ok; ++t)
-                if (code & (t ? kLive1 : kLive0)) ok = do_qk(t, s);
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+                if (ok && (code & (t ? kLive1 : kLive0))) ok = do_qk(t, s);
             if (!ok) break;
             tc_commit_if(leader, bar(C::kBarSlotEmpty + s));
             if (un.E == 1) tc_commit_if(leader, bar(kBarQEmpty));
@@ -362,15 +363,17 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
                 // Per tile: the next S first (it only needs the softmax to have read the
                 // current S), then P.V of the current entry.  Tile 0 runs ahead of tile 1
                 // (the softmax groups take turns), so tile 0 is served first.
-                for (int t = 0; t < 2 && ok; ++t) {
-                    if (next & (t ? kLive1 : kLive0)) ok = do_qk(t, ks);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (ok && (next & (t ? kLive1 : kLive0))) ok = do_qk(t, ks);
                     if (ok && (code & (t ? kLive1 : kLive0))) ok = do_pv(t, vs);
                 }
             } else {
                 // P_t lives in S_t: P.V of the current entry must be issued before the
                 // next Q K^T overwrites it.
-                for (int t = 0; t < 2 && ok; ++t) {
-                    if (code & (t ? kLive1 : kLive0)) ok = do_pv(t, vs);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (ok && (code & (t ? kLive1 : kLive0))) ok = do_pv(t, vs);
                     if (ok && (next & (t ? kLive1 : kLive0))) ok = do_qk(t, ks);
                 }
             }
@@ -383,6 +386,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
             code = next;
         }
         if (!ok) break;
+#pragma unroll
         for (int t = 0; t < 2; ++t)
             if (nl[t] > 0) ++of_cnt[t];
     }
