@@ -84,7 +84,7 @@ def read_peaks() -> dict:
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("attn_fwd.cu", "sm100_ptx.cuh", "fa_internal.h"):
+    for f in ("attn_fwd.cu", "fwd_common.cuh", "sm100_ptx.cuh", "fa_internal.h"):
         with open(os.path.join(ROOT, "block_sparse_masked_x128_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -12,6 +13,7 @@
 namespace {
 
 thread_local std::string g_last_error;
+std::atomic<int> g_stall_loads{0};
 
 fa_status_t fail(fa_status_t s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 fa_status_t fail(fa_status_t s, const char* fmt, ...) {
@@ -362,6 +364,7 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
     p.out_stride[2] = out->stride[2];
     p.lse = lse;
     p.status = m->status;
+    p.stall_loads = g_stall_loads.load(std::memory_order_relaxed);
 
     const int nsm = sm_count(dev);
     if (nsm <= 0) return fail(FA_ERR_CUDA, "could not read the SM count");
@@ -369,6 +372,12 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
     e = fa::launch_attn_fwd(p, (int)q->D, q->dtype == FA_DTYPE_BF16, (int)score_mod_kind, tq, tk, tv,
                             grid, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return ok();
+}
+
+// Test hook for failure detection (see the header): read by every later fa_forward.
+fa_status_t fa_debug_set_stall(int32_t enable) {
+    g_stall_loads.store(enable ? 1 : 0, std::memory_order_relaxed);
     return ok();
 }
 

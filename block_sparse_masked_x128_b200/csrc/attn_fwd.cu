@@ -30,23 +30,13 @@
 #include "fa_internal.h"
 #include "fa_trace.cuh"
 #include "sm100_ptx.cuh"
+#include "fwd_common.cuh"
 
 #ifdef FA_TRACE
 extern "C" int fa_debug_set_trace_buffer(void* device_ptr) {
     return (int)cudaMemcpyToSymbol(g_fa_trace, &device_ptr, sizeof(device_ptr));
 }
 #endif
-
-// Test hook for failure detection: while nonzero, every forward's producer warp stops after
-// the first unit's Q load, so the MMA warp's bounded wait for K runs out, the kernel unwinds
-// and the mask's status word reports the timeout.  Nothing faults, traps or hangs.
-static __device__ int g_fa_stall_loads = 0;
-
-extern "C" fa_status_t fa_debug_set_stall(int32_t enable) {
-    const int v = enable ? 1 : 0;
-    const cudaError_t e = cudaMemcpyToSymbol(g_fa_stall_loads, &v, sizeof(v));
-    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
 
 namespace fa {
 namespace {
@@ -60,15 +50,9 @@ constexpr int kRegsProducer = 104;
 constexpr int kRegsSoftmax = 200;
 static_assert(128 * kRegsProducer + 256 * kRegsSoftmax <= kThreadsFwd * kRegsAtLaunch,
               "register split exceeds the launched pool");
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;         // log2 of the largest P allowed
 
-// Barrier slots.
+// Barrier slots (kBarQFull = 0 and kBarQEmpty = 1 come with the producer).
 enum : int {
-    kBarQFull = 0,
-    kBarQEmpty = 1,
     kBarSFull = 2,    // + tile
     kBarPFull = 4,    // + tile
     kBarOFull = 6,    // + tile
@@ -76,7 +60,7 @@ enum : int {
     kBarSFree = 10,   // + tile: softmax has S in registers (separate-P layout only)
     kBarPVDone = 12,  // + tile: the tile's last P.V has completed (separate-P layout only)
     kBarDrain = 14,
-    kBarSlotFull = 15 // + stage, then slot-empty barriers follow
+    kBarSlotBase = 15 // + stage, then slot-empty barriers follow
 };
 
 template <int D>
@@ -84,6 +68,7 @@ struct Cfg {
     static constexpr int kTileBytes = kBlock * D * 2;
     static constexpr int kStages = (D == 64) ? 8 : 4;
     static constexpr int kChunks = D / 64;               // 128-byte-wide TMA boxes per row
+    static constexpr int kBarSlotFull = kBarSlotBase;
     static constexpr int kBarSlotEmpty = kBarSlotFull + kStages;
     static constexpr int kNumBars = kBarSlotEmpty + kStages;
     static constexpr int kBarOff = (2 + kStages) * kTileBytes;
@@ -104,149 +89,6 @@ struct Cfg {
         return kSepP ? 384u + (uint32_t)t * 64u : 256u + (uint32_t)t * (uint32_t)D;
     }
 };
-
-struct Unit {
-    int b, h, pair, E;
-    const int32_t* entries;
-};
-
-// The k-th unit of this CTA.  Units are in descending-cost order; rounds of gridDim.x
-// units are dealt alternately forwards and backwards over the CTAs ("snake" order), which
-// keeps the per-CTA sums of a longest-first list close to equal.
-__device__ __forceinline__ int unit_of_round(int k) {
-    const int G = (int)gridDim.x;
-    const int slot = (k & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-    return k * G + slot;
-}
-
-__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
-    const int BH = p.B * p.H;
-    const int r = u / BH, bh = u - r * BH;
-    const int b = bh / p.H, h = bh - b * p.H;
-    const int mb = (p.maskB == 1) ? 0 : b, mh = (p.maskH == 1) ? 0 : h;
-    const size_t sidx = (size_t)mb * p.maskH + mh;
-    Unit un;
-    un.b = b;
-    un.h = h;
-    un.pair = __ldg(p.sched_order + sidx * p.NP + r);
-    un.E = __ldg(p.sched_count + sidx * p.NP + un.pair);
-    un.entries = p.sched_entries + (sidx * p.NP + un.pair) * (size_t)p.KVB;
-    return un;
-}
-
-// Warp-collective reader of a unit's entry list: lane l caches entry base + l.
-// Indices passed to get() must not decrease.
-struct EntryReader {
-    const int32_t* ptr;
-    int E, base, val;
-    __device__ __forceinline__ void init(const int32_t* p, int n) {
-        ptr = p;
-        E = n;
-        base = -64;
-        val = 0;
-    }
-    __device__ __forceinline__ int get(int e) {
-        const int nb = e & ~31;
-        if (nb != base) {
-            base = nb;
-            const int idx = nb + (int)(threadIdx.x & 31);
-            val = idx < E ? __ldg(ptr + idx) : 0;
-        }
-        return __shfl_sync(kFullMask, val, e & 31);
-    }
-};
-
-__device__ __forceinline__ void count_live(const int32_t* entries, int E, int& n0, int& n1) {
-    int c0 = 0, c1 = 0;
-    for (int e = threadIdx.x & 31; e < E; e += 32) {
-        const int c = __ldg(entries + e);
-        c0 += (c & kLive0) ? 1 : 0;
-        c1 += (c & kLive1) ? 1 : 0;
-    }
-    n0 = __reduce_add_sync(kFullMask, c0);
-    n1 = __reduce_add_sync(kFullMask, c1);
-}
-
-// Wait without regard to the abort flag (used to drain in-flight copies on the way out).
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) break;
-    }
-    __syncwarp();
-}
-
-// ------------------------------------------------------------------ producer (warp 0)
-
-template <int D>
-__device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const CUtensorMap* tmk,
-                              const CUtensorMap* tmv, uint32_t sbase, uint32_t bars,
-                              volatile int* abort_flag) {
-    using C = Cfg<D>;
-    const uint32_t sQ = sbase, sKV = sbase + 2 * C::kTileBytes;
-    auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
-    auto wait = [&](int i, uint32_t par) {
-        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
-    };
-    const uint32_t leader = elect_one_lane();
-    if (leader) {
-        tma_prefetch_desc(tmq);
-        tma_prefetch_desc(tmk);
-        tma_prefetch_desc(tmv);
-    }
-    __syncwarp();
-    uint32_t kv_pos = 0, q_iter = 0;
-    bool ok = true;
-    const bool stall = *reinterpret_cast<volatile int*>(&g_fa_stall_loads) != 0;
-    FA_TRACE_DECL
-    for (int k = 0; ok; ++k) {
-        const int u = unit_of_round(k);
-        if (u >= p.n_units) break;
-        const Unit un = decode_unit(p, u);
-        if (un.E == 0) continue;
-        FA_TRACE_EV(0, 40);
-        if (!wait(kBarQEmpty, (q_iter & 1u) ^ 1u)) { ok = false; break; }
-        const int q0 = 2 * un.pair;
-        const int nq = (q0 + 1 < p.QB) ? 2 : 1;
-        mbar_arrive_expect_tx_if(leader, bar(kBarQFull), (uint32_t)(nq * C::kTileBytes));
-        for (int t = 0; t < nq; ++t)
-            for (int c = 0; c < C::kChunks; ++c)
-                tma_load_4d_if(leader, sQ + t * C::kTileBytes + c * 16384, tmq, bar(kBarQFull),
-                               c * 64, (q0 + t) * kBlock, un.h, un.b);
-        ++q_iter;
-        if (stall) {  // test hook: let Q land, then never load K or V
-            drain_wait(bar(kBarQFull), (q_iter - 1) & 1u);
-            return;
-        }
-        EntryReader er;
-        er.init(un.entries, un.E);
-        for (int e = 0; e < un.E && ok; ++e) {
-            const int j = er.get(e) & 0xFFFF;
-            for (int which = 0; which < 2; ++which) {
-                const int s = (int)(kv_pos % C::kStages);
-                const uint32_t ph = (kv_pos / C::kStages) & 1u;
-                FA_TRACE_EV(0, 30 + which);
-                if (!wait(C::kBarSlotEmpty + s, ph ^ 1u)) { ok = false; break; }
-                FA_TRACE_EV(0, 32 + which);
-                mbar_arrive_expect_tx_if(leader, bar(kBarSlotFull + s), (uint32_t)C::kTileBytes);
-                const CUtensorMap* tm = which ? tmv : tmk;
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_4d_if(leader, sKV + s * C::kTileBytes + c * 16384, tm,
-                                   bar(kBarSlotFull + s), c * 64, j * kBlock, un.h, un.b);
-                ++kv_pos;
-            }
-        }
-    }
-    if (!ok) {
-        // Let every copy already issued land before the CTA can exit.
-        const uint32_t n = kv_pos < (uint32_t)C::kStages ? kv_pos : (uint32_t)C::kStages;
-        for (uint32_t k = 0; k < n; ++k) {
-            const uint32_t pos = kv_pos - 1 - k;
-            drain_wait(bar(kBarSlotFull + (int)(pos % C::kStages)), (pos / C::kStages) & 1u);
-        }
-        if (q_iter > 0) drain_wait(bar(kBarQFull), (q_iter - 1) & 1u);
-    }
-}
 
 // ------------------------------------------------------------------ MMA issuer (warp 1)
 
@@ -340,7 +182,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
         {   // S for entry 0
             const uint32_t pos = kbase;
             const int s = (int)(pos % C::kStages);
-            if (!wait(kBarSlotFull + s, (pos / C::kStages) & 1u)) { ok = false; break; }
+            if (!wait(C::kBarSlotFull + s, (pos / C::kStages) & 1u)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int t = 0; t < 2; ++t)
@@ -355,8 +197,8 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
             const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u, kpos = vpos + 1u;
             const int vs = (int)(vpos % C::kStages), ks = (int)(kpos % C::kStages);
             FA_TRACE_EV(1, 22);
-            if (!wait(kBarSlotFull + vs, (vpos / C::kStages) & 1u)) { ok = false; break; }
-            if (has_next && !wait(kBarSlotFull + ks, (kpos / C::kStages) & 1u)) { ok = false; break; }
+            if (!wait(C::kBarSlotFull + vs, (vpos / C::kStages) & 1u)) { ok = false; break; }
+            if (has_next && !wait(C::kBarSlotFull + ks, (kpos / C::kStages) & 1u)) { ok = false; break; }
             FA_TRACE_EV(1, 23);
             tc_fence_after();
             if constexpr (C::kSepP) {
@@ -431,15 +273,6 @@ __device__ __forceinline__ float2 softmax_p_row(const float2 (&x)[64], float2 nb
         tmem_st_32x32b_x16(tP + chunk * 16, pk);
     }
     return __fadd2_rn(__fadd2_rn(rs[0], rs[1]), __fadd2_rn(rs[2], rs[3]));
-}
-
-template <int D, bool BF16>
-__device__ __forceinline__ void store_row_zero(const FwdParams& p, const Unit& un, int q) {
-    uint16_t* o = reinterpret_cast<uint16_t*>(p.out) + un.b * p.out_stride[0] +
-                  un.h * p.out_stride[1] + (int64_t)q * p.out_stride[2];
-#pragma unroll
-    for (int d = 0; d < D; d += 8) *reinterpret_cast<uint4*>(o + d) = make_uint4(0, 0, 0, 0);
-    if (p.lse) p.lse[((int64_t)un.b * p.H + un.h) * p.Q_LEN + q] = -INFINITY;
 }
 
 template <int D, bool BF16, int SCORE>
@@ -702,7 +535,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
         }
         mbar_init(bars + 8u * kBarDrain, 1);
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(bars + 8u * (kBarSlotFull + s), 1);
+            mbar_init(bars + 8u * (C::kBarSlotFull + s), 1);
             mbar_init(bars + 8u * (C::kBarSlotEmpty + s), 1);
         }
         *abort_flag = 0;
@@ -722,7 +555,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
     if (warp < 4) {
         regs_dec<kRegsProducer>();
         if (warp == 0) {
-            producer_role<D>(p, &tmq, &tmk, &tmv, sbase, bars, abort_flag);
+            producer_role<Cfg<D>>(p, &tmq, &tmk, &tmv, sbase, bars, abort_flag);
         } else if (warp == 1) {
             mma_role<D, BF16>(p, sbase, bars, tmem, abort_flag);
         }

@@ -53,6 +53,7 @@ struct FwdParams {
     int64_t out_stride[3];        // B, H, S strides in elements (D stride is 1)
     float* lse;                   // [B][H][Q_LEN] or null
     int32_t* status;              // device status word (1 = a bounded wait ran out)
+    int32_t stall_loads;          // test hook: the TMA warp stops after the first Q tiles
 };
 
 cudaError_t launch_mask_build(const MaskSpec& spec, int separate_full, int maskBH, int NP,

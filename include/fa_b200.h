@@ -209,13 +209,12 @@ const char* fa_last_error_message(void);
 
 /*
  * Test hook for failure detection (no counterpart on the pages).  While `enable` is nonzero,
- * the TMA warp of every subsequent fa_forward on the current device loads only the first
+ * the TMA warp of every fa_forward launched afterwards (process-wide) loads only the first
  * query tiles and then stops, so the MMA warp's bounded wait for K runs past its limit
  * (about two seconds), every role of the kernel unwinds and releases its tensor memory,
  * and the mask's status word is set: fa_get_device_status then returns FA_ERR_TIMEOUT.
- * The outputs of such a call are unspecified.  Pass 0 to restore normal operation.  Device
- * global state: not for use while other threads run forwards on the same device.
- * Returns FA_OK or FA_ERR_CUDA.
+ * The outputs of such a call are unspecified.  Pass 0 to restore normal operation.  Process
+ * global state: not for use while other threads launch forwards.  Returns FA_OK.
  */
 fa_status_t fa_debug_set_stall(int32_t enable);
 
