@@ -404,7 +404,7 @@ def run_reference(args, w: wl.Workload, world: int, rank: int) -> dict:
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference", "config": config_dict(w, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"{tot_rows} query rows ({rows} per step) of {w.name}"},
+                             "sample": f"{tot_rows} query rows of {w.name} in {rows}-row chunks, about {per_step:.2g} s per step"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
