@@ -16,7 +16,11 @@
 //   2. schedule_kernel: one CTA per work unit (a pair of adjacent query blocks) merges
 //      the two tiles' partial and full lists into one list of kv blocks, nearest first
 //      (descending), with per-tile live/full flags, so the forward kernel loads each K/V
-//      tile once for both query tiles.  The unit's cost is the number of live tiles.
+//      tile once for both query tiles.  The unit's cost estimates its forward time in
+//      quarter entries: an entry with both tiles live costs 4 (the two softmax groups run
+//      side by side), an entry with one live tile 3 (one group runs alone, faster per tile
+//      but not twice as fast), plus 2 for the unit's prologue and epilogue; with L live
+//      tiles over n entries that is L + 2n + 2.
 //   3. lpt_order_kernel: ranks the units of each stored (b, h) by descending cost (ties
 //      by index) so the persistent forward kernel hands the longest units out first.
 #include <climits>
@@ -239,7 +243,7 @@ schedule_kernel(int QB, int KVB, int NP, const int32_t* __restrict__ kv_num,
     }
     if (tid == 0) {
         sched_count[unit] = cnt;
-        sched_cost[unit] = l0 + l1;
+        sched_cost[unit] = l0 + l1 + 2 * cnt + 2;
     }
 }
 
