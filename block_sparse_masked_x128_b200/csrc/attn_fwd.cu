@@ -60,7 +60,9 @@ enum : int {
     kBarSFree = 10,   // + tile: softmax has S in registers (separate-P layout only)
     kBarPVDone = 12,  // + tile: the tile's last P.V has completed (separate-P layout only)
     kBarDrain = 14,
-    kBarSlotBase = 15 // + stage, then slot-empty barriers follow
+    kBarUnitFull = 15,  // + unit-ring slot (2)
+    kBarUnitEmpty = 17, // + unit-ring slot (2)
+    kBarSlotBase = 19   // + stage, then slot-empty barriers follow
 };
 
 template <int D>
@@ -68,11 +70,14 @@ struct Cfg {
     static constexpr int kTileBytes = kBlock * D * 2;
     static constexpr int kStages = (D == 64) ? 8 : 4;
     static constexpr int kChunks = D / 64;               // 128-byte-wide TMA boxes per row
+    static constexpr int kBarUFull = kBarUnitFull;
+    static constexpr int kBarUEmpty = kBarUnitEmpty;
     static constexpr int kBarSlotFull = kBarSlotBase;
     static constexpr int kBarSlotEmpty = kBarSlotFull + kStages;
     static constexpr int kNumBars = kBarSlotEmpty + kStages;
     static constexpr int kBarOff = (2 + kStages) * kTileBytes;
-    static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + alignment slack
+    // After the barriers: TMEM address, abort flag, the two unit-ring slots.
+    static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;  // + alignment slack
     // TMEM columns.  At D = 64 everything fits apart: S0 S1 (128 each), P0 P1 (64 each),
     // O0 O1 (64 each) = 512, so the next Q K^T can overwrite S while P is still being
     // computed.  At D = 128, P_t is written over the first 64 columns of S_t.
@@ -94,7 +99,7 @@ struct Cfg {
 
 template <int D, bool BF16>
 __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
-                         volatile int* abort_flag) {
+                         const volatile int* ring, volatile int* abort_flag) {
     using C = Cfg<D>;
     const uint32_t leader = elect_one_lane();
     const uint32_t sQ = sbase, sKV = sbase + 2 * C::kTileBytes;
@@ -149,9 +154,10 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
         tc_commit_if(leader, bar(kBarSFull + t));
         return true;
     };
-    for (int k = 0; ok; ++k) {
-        const int u = unit_of_round(k);
-        if (u >= p.n_units) break;
+    uint32_t u_iter = 0;
+    for (;;) {
+        const int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, ok);
+        if (u < 0) break;
         const Unit un = decode_unit(p, u);
         if (un.E == 0) continue;
         int nl[2];
@@ -277,7 +283,7 @@ __device__ __forceinline__ float2 softmax_p_row(const float2 (&x)[64], float2 nb
 
 template <int D, bool BF16, int SCORE>
 __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t tmem,
-                             volatile int* abort_flag) {
+                             const volatile int* ring, volatile int* abort_flag) {
     using C = Cfg<D>;
     const int wq = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant this warp may access
     const int lane = threadIdx.x & 31;
@@ -299,9 +305,11 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
     const int tslot = 2 + (int)(threadIdx.x >> 5) - 4;  // one trace slot per softmax warp
     FA_TRACE_DECL
     (void)tslot;
-    for (int k = 0;; ++k) {
-        const int u = unit_of_round(k);
-        if (u >= p.n_units) break;
+    uint32_t u_iter = 0;
+    for (;;) {
+        bool taken = true;
+        const int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, taken);
+        if (u < 0) return;
         const Unit un = decode_unit(p, u);
         const int qblk = 2 * un.pair + t;
         int nl0 = 0, nl1 = 0;
@@ -520,6 +528,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
     const uint32_t bars = sbase + C::kBarOff;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
     const int warp = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
@@ -534,6 +543,10 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
             mbar_init(bars + 8u * (kBarPVDone + t), 1);
         }
         mbar_init(bars + 8u * kBarDrain, 1);
+        for (int r = 0; r < kUnitRing; ++r) {
+            mbar_init(bars + 8u * (C::kBarUFull + r), 1);    // the TMA warp publishes
+            mbar_init(bars + 8u * (C::kBarUEmpty + r), 9);   // the MMA warp + 8 softmax warps
+        }
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(bars + 8u * (C::kBarSlotFull + s), 1);
             mbar_init(bars + 8u * (C::kBarSlotEmpty + s), 1);
@@ -555,13 +568,13 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
     if (warp < 4) {
         regs_dec<kRegsProducer>();
         if (warp == 0) {
-            producer_role<Cfg<D>>(p, &tmq, &tmk, &tmv, sbase, bars, abort_flag);
+            producer_role<Cfg<D>>(p, &tmq, &tmk, &tmv, sbase, bars, ring, abort_flag);
         } else if (warp == 1) {
-            mma_role<D, BF16>(p, sbase, bars, tmem, abort_flag);
+            mma_role<D, BF16>(p, sbase, bars, tmem, ring, abort_flag);
         }
     } else {
         regs_inc<kRegsSoftmax>();
-        softmax_role<D, BF16, SCORE>(p, (warp - 4) >> 2, bars, tmem, abort_flag);
+        softmax_role<D, BF16, SCORE>(p, (warp - 4) >> 2, bars, tmem, ring, abort_flag);
     }
     tc_fence_before();
     __syncthreads();

@@ -53,6 +53,7 @@ struct FwdParams {
     int64_t out_stride[3];        // B, H, S strides in elements (D stride is 1)
     float* lse;                   // [B][H][Q_LEN] or null
     int32_t* status;              // device status word (1 = a bounded wait ran out)
+    int32_t* sched_ctr;           // [0] next unit to hand out, [1] CTAs done; both 0 between launches
     int32_t stall_loads;          // test hook: the TMA warp stops after the first Q tiles
 };
 
@@ -97,4 +98,5 @@ struct fa_block_mask {
     int32_t* sched_entries;
     int32_t* sched_order;
     int32_t* status;
+    int32_t* sched_ctr;       // two words after the status word
 };

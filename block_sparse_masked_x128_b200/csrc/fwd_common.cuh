@@ -8,7 +8,8 @@
 // live/full flags of the two query tiles (kLive0, kFull0, kLive1, kFull1).  The producer
 // loads both Q tiles of a unit, then K_j and V_j of every entry into a ring of shared-memory
 // stages; a configuration class C supplies the tile size, the ring depth and the barrier
-// slots (kBarQFull / kBarQEmpty at 0 / 1, C::kBarSlotFull and C::kBarSlotEmpty per stage).
+// slots (kBarQFull / kBarQEmpty at 0 / 1, C::kBarSlotFull and C::kBarSlotEmpty per stage,
+// C::kBarUFull and C::kBarUEmpty per slot of the unit ring).
 #pragma once
 
 #include "fa_internal.h"
@@ -29,15 +30,6 @@ struct Unit {
     int b, h, pair, E;
     const int32_t* entries;
 };
-
-// The k-th unit of this CTA.  Units are in descending-cost order; rounds of gridDim.x
-// units are dealt alternately forwards and backwards over the CTAs ("snake" order), which
-// keeps the per-CTA sums of a longest-first list close to equal.
-__device__ __forceinline__ int unit_of_round(int k) {
-    const int G = (int)gridDim.x;
-    const int slot = (k & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-    return k * G + slot;
-}
 
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     const int BH = p.B * p.H;
@@ -87,6 +79,31 @@ __device__ __forceinline__ void count_live(const int32_t* entries, int E, int& n
     n1 = __reduce_add_sync(kFullMask, c1);
 }
 
+// Units are handed out at run time, longest first: the TMA warp of each CTA takes the next
+// index from a global counter (atomicAdd on sched_ctr[0]) when it is ready for another unit
+// and publishes it to the MMA and softmax warps through a two-slot ring in shared memory
+// (C::kBarUFull / C::kBarUEmpty per slot; -1 ends the sequence).  A CTA that finishes early
+// simply takes more units, so the per-CTA work evens out whatever the units really cost.
+constexpr int kUnitRing = 2;
+
+// Consumer side: the next unit of this CTA, -1 when there is none; ok turns false when the
+// bounded wait gave up.  Called by every lane of a warp.
+template <class C>
+__device__ __forceinline__ int take_unit(const FwdParams& p, uint32_t bars, const volatile int* ring,
+                                         uint32_t& u_iter, volatile int* abort_flag, bool& ok) {
+    const int slot = (int)(u_iter % kUnitRing);
+    const uint32_t par = (u_iter / kUnitRing) & 1u;
+    if (!mbar_wait_bounded(bars + 8u * (uint32_t)(C::kBarUFull + slot), par, abort_flag, p.status,
+                           kWaitLimitNs)) {
+        ok = false;
+        return -1;
+    }
+    const int u = ring[slot];
+    mbar_arrive_warp(bars + 8u * (uint32_t)(C::kBarUEmpty + slot));
+    ++u_iter;
+    return u;
+}
+
 // Wait without regard to the abort flag (used to drain in-flight copies on the way out).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
     const uint64_t t0 = global_timer_ns();
@@ -101,7 +118,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 template <class C>
 __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const CUtensorMap* tmk,
                               const CUtensorMap* tmv, uint32_t sbase, uint32_t bars,
-                              volatile int* abort_flag) {
+                              volatile int* ring, volatile int* abort_flag) {
     const uint32_t sQ = sbase, sKV = sbase + 2 * C::kTileBytes;
     auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
     auto wait = [&](int i, uint32_t par) {
@@ -114,13 +131,42 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
         tma_prefetch_desc(tmv);
     }
     __syncwarp();
-    uint32_t kv_pos = 0, q_iter = 0;
+    const int leader_lane = __ffs(__ballot_sync(kFullMask, leader != 0)) - 1;
+    // Done taking units: the last CTA to get here resets the counters for the next launch
+    // (every CTA gets here, also after a timeout, because every wait is bounded).
+    auto finish = [&]() {
+        if (leader) {
+            __threadfence();
+            if (atomicAdd(p.sched_ctr + 1, 1) == (int)gridDim.x - 1) {
+                p.sched_ctr[0] = 0;
+                p.sched_ctr[1] = 0;
+                __threadfence();
+            }
+        }
+        __syncwarp();
+    };
+    uint32_t kv_pos = 0, q_iter = 0, u_iter = 0;
     bool ok = true;
     const bool stall = p.stall_loads != 0;
     FA_TRACE_DECL
-    for (int k = 0; ok; ++k) {
-        const int u = unit_of_round(k);
-        if (u >= p.n_units) break;
+    for (;;) {
+        int u = -1;
+        if (leader) {
+            const int v = atomicAdd(p.sched_ctr, 1);
+            u = v < p.n_units ? v : -1;
+        }
+        u = __shfl_sync(kFullMask, u, leader_lane);
+        {   // publish it to the MMA and softmax warps
+            const int slot = (int)(u_iter % kUnitRing);
+            if (!wait(C::kBarUEmpty + slot, ((u_iter / kUnitRing) & 1u) ^ 1u)) { ok = false; break; }
+            if (leader) {
+                ring[slot] = u;
+                mbar_arrive(bar(C::kBarUFull + slot));
+            }
+            __syncwarp();
+            ++u_iter;
+        }
+        if (u < 0) break;
         const Unit un = decode_unit(p, u);
         if (un.E == 0) continue;
         FA_TRACE_EV(0, 40);
@@ -135,6 +181,7 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
         ++q_iter;
         if (stall) {  // test hook: let Q land, then never load K or V
             drain_wait(bar(kBarQFull), (q_iter - 1) & 1u);
+            finish();
             return;
         }
         EntryReader er;
@@ -165,6 +212,7 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
         }
         if (q_iter > 0) drain_wait(bar(kBarQFull), (q_iter - 1) & 1u);
     }
+    finish();
 }
 
 // A query row with no live key: O = 0 and lse = -inf.
