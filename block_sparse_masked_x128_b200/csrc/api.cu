@@ -177,7 +177,9 @@ fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* par
     const size_t o_dst = take(has_doc ? (size_t)(QB > KVB ? QB : KVB) * 3 * 4 : 0);
     const size_t o_sc = take(BH * NP * 4), o_scost = take(BH * NP * 4);
     const size_t o_se = take(BH * NP * KVB * 4), o_so = take(BH * NP * 4);
-    const size_t o_status = take(16);  // status word, then the forward's unit counters
+    // Status word, then the forward's unit counters (two words per slot), all zero.
+    const size_t ctr_bytes = 4 + (size_t)fa::kSchedCtrSlots * 8;
+    const size_t o_status = take(ctr_bytes);
     void* base = nullptr;
     e = cudaMalloc(&base, off);
     if (e != cudaSuccess) {
@@ -217,7 +219,7 @@ fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* par
         delete m;
         return cuda_fail(err, what);
     };
-    if ((e = cudaMemsetAsync(m->status, 0, 16, st)) != cudaSuccess) return bail(e, "cudaMemsetAsync");
+    if ((e = cudaMemsetAsync(m->status, 0, ctr_bytes, st)) != cudaSuccess) return bail(e, "cudaMemsetAsync");
     if (has_doc &&
         (e = cudaMemcpyAsync(m->doc, params->doc_id, (size_t)KV_LEN * 4, cudaMemcpyDefault, st)) !=
             cudaSuccess)
@@ -276,8 +278,7 @@ fa_status_t fa_get_device_status(const fa_block_mask_t* m, void* stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
     if (h != 0) {
-        // Clear the status word and, after an aborted forward, the unit counters too.
-        e = cudaMemsetAsync(m->status, 0, 16, st);
+        e = cudaMemsetAsync(m->status, 0, 4, st);
         if (e == cudaSuccess) e = cudaStreamSynchronize(st);
         if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
         return fail(FA_ERR_TIMEOUT, "a device-side wait ran past its limit (status %d)", h);
@@ -366,7 +367,13 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
     p.out_stride[2] = out->stride[2];
     p.lse = lse;
     p.status = m->status;
-    p.sched_ctr = m->sched_ctr;
+    {
+        // A pair of unit counters of its own for this launch (the kernel's last CTA returns
+        // them to zero, also after a timeout).
+        fa_block_mask_t* mm = const_cast<fa_block_mask_t*>(m);
+        const uint32_t slot = mm->next_ctr.fetch_add(1, std::memory_order_relaxed) % fa::kSchedCtrSlots;
+        p.sched_ctr = m->sched_ctr + 2 * slot;
+    }
     p.stall_loads = g_stall_loads.load(std::memory_order_relaxed);
 
     const int nsm = sm_count(dev);

@@ -1,6 +1,8 @@
 // fa_internal.h -- structures shared by the host API (api.cu) and the kernels.
 #pragma once
 
+#include <atomic>
+
 #include <cstddef>
 #include <cstdint>
 
@@ -77,6 +79,10 @@ cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, int score_kind
                             const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             int grid, cudaStream_t stream);
 
+// Counter pairs per mask for the forward's run-time unit hand-out: each launch takes the
+// next pair, so up to this many forwards may run at once on one mask.
+constexpr int kSchedCtrSlots = 64;
+
 }  // namespace fa
 
 struct fa_block_mask {
@@ -98,5 +104,6 @@ struct fa_block_mask {
     int32_t* sched_entries;
     int32_t* sched_order;
     int32_t* status;
-    int32_t* sched_ctr;       // two words after the status word
+    int32_t* sched_ctr;       // fa::kSchedCtrSlots pairs of unit counters after the status word
+    std::atomic<uint32_t> next_ctr{0};  // round-robin pick of a counter pair per forward
 };

@@ -25,8 +25,9 @@
  *     argument checks happen before any launch; on an error nothing is launched and
  *     no output is written.  fa_last_error_message() gives a one-line reason.
  *   - Library objects are not thread-safe against concurrent destroy; concurrent
- *     fa_forward calls on one mask from different streams are allowed (the mask is
- *     read-only for them).
+ *     fa_forward calls on one mask from different streams are allowed, up to 64 in
+ *     flight at once (the lists are read-only for them; each launch takes the next of
+ *     the mask's 64 pairs of work-distribution counters, which its kernel leaves zero).
  */
 #ifndef FA_B200_H
 #define FA_B200_H

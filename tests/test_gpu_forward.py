@@ -208,3 +208,41 @@ def test_lse_may_be_omitted_and_runs_are_deterministic():
     assert torch.equal(o1, o2)
     o3, l3 = fa.flex_attention(q, k, v, bm)
     assert torch.equal(o2, o3) and torch.equal(l2, l3)
+
+
+def test_forwards_on_one_mask_from_two_streams():
+    # Each launch takes its own pair of the mask's work-distribution counters, so forwards
+    # that share a mask may overlap on different streams.
+    fa = fa_module()
+    g = torch.Generator().manual_seed(12)
+    q, k, v = (torch.randn(1, 8, 2048, 64, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    bm = gpu_block_mask(C, None, None, 2048, 2048)
+    o_ref, l_ref = fa.flex_attention(q, k, v, bm)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for i in range(8):
+        st = streams[i % 2]
+        with torch.cuda.stream(st):
+            out = torch.empty_like(q)
+            lse = torch.empty(1, 8, 2048, device="cuda")
+            fa.flex_attention(q, k, v, bm, out=out, lse=lse, stream=st)
+            outs.append((out, lse))
+    torch.cuda.synchronize()
+    assert bm.device_status() == fa.FA_OK
+    for out, lse in outs:
+        assert torch.equal(out, o_ref) and torch.equal(lse, l_ref)
+
+
+def test_many_forwards_reuse_the_counters():
+    # More launches than the mask has counter pairs: every pair must come back zeroed.
+    fa = fa_module()
+    w = wl.WORKLOADS[3].scaled(S=1024, H=2)
+    q, k, v = (t.cuda() for t in wl.make_qkv(w))
+    doc = wl.make_doc_ids(w)
+    bm = gpu_block_mask(w.mask_kind, None, None, w.S, w.S, 0, doc)
+    o_ref, l_ref = fa.flex_attention(q, k, v, bm)
+    for _ in range(70):
+        o, l = fa.flex_attention(q, k, v, bm)
+        assert torch.equal(o, o_ref) and torch.equal(l, l_ref)
+    assert bm.device_status() == fa.FA_OK
