@@ -175,7 +175,7 @@ fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* par
     const bool has_doc = (mask_kind & FA_MASK_DOCUMENT) != 0;
     const size_t o_doc = take(has_doc ? (size_t)KV_LEN * 4 : 0);
     const size_t o_dst = take(has_doc ? (size_t)(QB > KVB ? QB : KVB) * 3 * 4 : 0);
-    const size_t o_sc = take(BH * NP * 4), o_scost = take(BH * NP * 4);
+    const size_t o_sc = take(BH * NP * 8), o_scost = take(BH * NP * 4);
     const size_t o_se = take(BH * NP * KVB * 4), o_so = take(BH * NP * 4);
     // Status word, then the forward's unit counters (two words per slot), all zero.
     const size_t ctr_bytes = 4 + (size_t)fa::kSchedCtrSlots * 8;

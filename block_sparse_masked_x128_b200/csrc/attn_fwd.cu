@@ -160,8 +160,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
         if (u < 0) break;
         const Unit un = decode_unit(p, u);
         if (un.E == 0) continue;
-        int nl[2];
-        count_live(un.entries, un.E, nl[0], nl[1]);
+        const int nl[2] = {un.nl0, un.nl1};
         if (!wait(kBarQFull, q_iter & 1u)) { ok = false; break; }
         ++q_iter;
         tc_fence_after();
@@ -306,18 +305,18 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
     FA_TRACE_DECL
     (void)tslot;
     uint32_t u_iter = 0;
+    bool taken = true;
+    // The next unit is taken before this unit's epilogue waits for O, so the ring handshake
+    // and the schedule reads overlap the last P.V instead of following it.
+    int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, taken);
     for (;;) {
-        bool taken = true;
-        const int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, taken);
         if (u < 0) return;
         const Unit un = decode_unit(p, u);
         const int qblk = 2 * un.pair + t;
-        int nl0 = 0, nl1 = 0;
-        if (un.E > 0) count_live(un.entries, un.E, nl0, nl1);
-        const int nl = t ? nl1 : nl0;
-        if (qblk >= p.QB) continue;
-        if (nl == 0) {
-            store_row_zero<D, BF16>(p, un, qblk * kBlock + row);
+        const int nl = t ? un.nl1 : un.nl0;
+        if (qblk >= p.QB || nl == 0) {
+            if (qblk < p.QB) store_row_zero<D, BF16>(p, un, qblk * kBlock + row);
+            u = take_unit<C>(p, bars, ring, u_iter, abort_flag, taken);
             continue;
         }
         const int q = qblk * kBlock + row;
@@ -482,6 +481,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             ++done;
         }
         if (!ok) return;
+        u = take_unit<C>(p, bars, ring, u_iter, abort_flag, taken);
         // Epilogue: O / l in the output dtype, and the natural-log lse.
         FA_TRACE_EV(tslot, 7);
         if (!wait(kBarOFull + t, of_cnt & 1u)) return;

@@ -43,7 +43,7 @@ struct FwdParams {
     uint32_t score_kind;
     const int32_t* doc_id;
     const int32_t* sched_order;   // [maskB*maskH][NP]  pairs by descending cost
-    const int32_t* sched_count;   // [maskB*maskH][NP]  entries per pair
+    const int32_t* sched_count;   // [maskB*maskH][NP][2]  entries; live tiles t0 | t1 << 16
     const int32_t* sched_entries; // [maskB*maskH][NP][KVB]
     float scale;                  // multiplies q k^T
     float scale_log2;             // scale * log2(e)

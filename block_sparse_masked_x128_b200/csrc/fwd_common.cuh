@@ -28,6 +28,7 @@ constexpr int kBarQEmpty = 1;
 
 struct Unit {
     int b, h, pair, E;
+    int nl0, nl1;  // live tiles of query tile 0 and 1
     const int32_t* entries;
 };
 
@@ -41,7 +42,10 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     un.b = b;
     un.h = h;
     un.pair = __ldg(p.sched_order + sidx * p.NP + r);
-    un.E = __ldg(p.sched_count + sidx * p.NP + un.pair);
+    const int2 c = __ldg(reinterpret_cast<const int2*>(p.sched_count) + sidx * p.NP + un.pair);
+    un.E = c.x;
+    un.nl0 = c.y & 0xFFFF;
+    un.nl1 = (int)((unsigned)c.y >> 16);
     un.entries = p.sched_entries + (sidx * p.NP + un.pair) * (size_t)p.KVB;
     return un;
 }
@@ -67,17 +71,6 @@ struct EntryReader {
         return __shfl_sync(kFullMask, val, e & 31);
     }
 };
-
-__device__ __forceinline__ void count_live(const int32_t* entries, int E, int& n0, int& n1) {
-    int c0 = 0, c1 = 0;
-    for (int e = threadIdx.x & 31; e < E; e += 32) {
-        const int c = __ldg(entries + e);
-        c0 += (c & kLive0) ? 1 : 0;
-        c1 += (c & kLive1) ? 1 : 0;
-    }
-    n0 = __reduce_add_sync(kFullMask, c0);
-    n1 = __reduce_add_sync(kFullMask, c1);
-}
 
 // Units are handed out at run time, longest first: the TMA warp of each CTA takes the next
 // index from a global counter (atomicAdd on sched_ctr[0]) when it is ready for another unit

@@ -242,7 +242,8 @@ schedule_kernel(int QB, int KVB, int NP, const int32_t* __restrict__ kv_num,
         __syncthreads();
     }
     if (tid == 0) {
-        sched_count[unit] = cnt;
+        sched_count[2 * unit] = cnt;
+        sched_count[2 * unit + 1] = l0 | (l1 << 16);
         sched_cost[unit] = l0 + l1 + 2 * cnt + 2;
     }
 }
