@@ -173,7 +173,7 @@ def test_per_head_mask_equals_broadcast_mask():
 
 
 @pytest.mark.parametrize("score_kind", [wl.SCORE_SOFTCAP, wl.SCORE_ALIBI, wl.SCORE_SOFTCAP | wl.SCORE_ALIBI])
-@pytest.mark.parametrize("D,dtype", [(64, "fp16"), (128, "bf16")])
+@pytest.mark.parametrize("D,dtype", [(64, "fp16"), (64, "bf16"), (128, "bf16"), (128, "fp16")])
 def test_score_mods(score_kind, D, dtype):
     w = wl.Workload("score_mods", B=1, H=4, S=768, D=D, dtype=dtype, mask_kind=C,
                     score_kind=score_kind, softcap=5.0, seed=23)
@@ -246,3 +246,16 @@ def test_many_forwards_reuse_the_counters():
         o, l = fa.flex_attention(q, k, v, bm)
         assert torch.equal(o, o_ref) and torch.equal(l, l_ref)
     assert bm.device_status() == fa.FA_OK
+
+
+@pytest.mark.parametrize("kind,window,score_kind", [(C, 0, wl.SCORE_NONE),
+                                                    (C | SW, 4096, wl.SCORE_SOFTCAP | wl.SCORE_ALIBI)])
+def test_long_sequence_sampled_rows(kind, window, score_kind):
+    # 131072 positions: 1024 blocks per side, units of up to 1024 entries.
+    w = wl.Workload("long", B=1, H=1, S=131072, D=64, dtype="bf16", mask_kind=kind, window=window,
+                    score_kind=score_kind, softcap=30.0, seed=25)
+    q, k, v = wl.make_qkv(w)
+    out, lse, _ = run_gpu(w, q, k, v)
+    rows = _sample_rows(w.S, w.seed, n_random=6)
+    O, L = run_oracle(w, q, k, v, rows=rows)
+    compare(out, lse, O, L, rows=rows)
