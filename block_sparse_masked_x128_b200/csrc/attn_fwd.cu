@@ -280,10 +280,16 @@ __device__ __forceinline__ float2 softmax_p_row(const float2 (&x)[64], float2 nb
     return __fadd2_rn(__fadd2_rn(rs[0], rs[1]), __fadd2_rn(rs[2], rs[3]));
 }
 
-template <int D, bool BF16, int SCORE>
+// VAR = score_mod bits (FA_SCORE_*) | kVarDocument when the mask has a document predicate:
+// both are compile-time, so kernels without them carry none of their registers.
+constexpr int kVarDocument = 4;
+
+template <int D, bool BF16, int VAR>
 __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t tmem,
                              const volatile int* ring, volatile int* abort_flag) {
     using C = Cfg<D>;
+    constexpr int SCORE = VAR & (FA_SCORE_SOFTCAP | FA_SCORE_ALIBI);
+    constexpr bool kDoc = (VAR & kVarDocument) != 0;
     const int wq = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant this warp may access
     const int lane = threadIdx.x & 31;
     const int row = wq * 32 + lane;
@@ -398,7 +404,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                 int lo = 0, hi = kBlock - 1;
                 if (p.mask_kind & (FA_MASK_CAUSAL | FA_MASK_SLIDING_WINDOW)) hi = min(hi, q - kv0);
                 if (p.mask_kind & FA_MASK_SLIDING_WINDOW) lo = max(lo, q - p.window + 1 - kv0);
-                if (p.mask_kind & FA_MASK_DOCUMENT) {
+                if constexpr (kDoc) {
                     const int dq = __ldg(p.doc_id + q);
                     const int4* dk = reinterpret_cast<const int4*>(p.doc_id + kv0);
 #pragma unroll
@@ -516,7 +522,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
 
 // ------------------------------------------------------------------ kernel
 
-template <int D, bool BF16, int SCORE>
+template <int D, bool BF16, int VAR>
 __global__ void __launch_bounds__(kThreadsFwd, 1)
 attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tmq,
                 const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
@@ -574,7 +580,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
         }
     } else {
         regs_inc<kRegsSoftmax>();
-        softmax_role<D, BF16, SCORE>(p, (warp - 4) >> 2, bars, tmem, ring, abort_flag);
+        softmax_role<D, BF16, VAR>(p, (warp - 4) >> 2, bars, tmem, ring, abort_flag);
     }
     tc_fence_before();
     __syncthreads();
@@ -582,10 +588,10 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
     if (warp == 2) tmem_dealloc(tmem, 512);
 }
 
-template <int D, bool BF16, int SCORE>
+template <int D, bool BF16, int VAR>
 cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                      const CUtensorMap& tv, int grid, cudaStream_t stream) {
-    auto kern = attn_fwd_kernel<D, BF16, SCORE>;
+    auto kern = attn_fwd_kernel<D, BF16, VAR>;
     // setmaxnreg.inc waits for registers from the launched pool; refuse to launch a build
     // whose per-thread register count would make that pool smaller than the split needs.
     cudaFuncAttributes attr;
@@ -603,10 +609,12 @@ cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMa
 cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, int score_kind,
                             const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             int grid, cudaStream_t stream) {
-#define FA_CASE(DD, BB, SS)                                                 \
-    if (D == DD && bf16 == BB && score_kind == SS)                          \
-        return launch_t<DD, BB, SS>(p, tq, tk, tv, grid, stream);
-#define FA_CASES(DD, BB) FA_CASE(DD, BB, 0) FA_CASE(DD, BB, 1) FA_CASE(DD, BB, 2) FA_CASE(DD, BB, 3)
+    const int var = score_kind | ((p.mask_kind & FA_MASK_DOCUMENT) ? kVarDocument : 0);
+#define FA_CASE(DD, BB, VV)                                                 \
+    if (D == DD && bf16 == BB && var == VV)                                 \
+        return launch_t<DD, BB, VV>(p, tq, tk, tv, grid, stream);
+#define FA_CASES(DD, BB) FA_CASE(DD, BB, 0) FA_CASE(DD, BB, 1) FA_CASE(DD, BB, 2) FA_CASE(DD, BB, 3) \
+    FA_CASE(DD, BB, 4) FA_CASE(DD, BB, 5) FA_CASE(DD, BB, 6) FA_CASE(DD, BB, 7)
     FA_CASES(64, true)
     FA_CASES(64, false)
     FA_CASES(128, true)
