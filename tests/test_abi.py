@@ -125,3 +125,37 @@ def test_python_binding_raises_fa_error(fa):
     with pytest.raises(fa.FaError) as ei:
         fa.fa_create_block_mask(1, None, 0, 0, 256, 256, BLOCK_SIZE=64, stream=0)
     assert ei.value.status == fa.FA_ERR_UNSUPPORTED
+
+
+def _header_constants():
+    text = open(os.path.join(ROOT, "include", "fa_b200.h")).read()
+    consts = {n: int(v) for n, v in re.findall(r"#define\s+(FA_[A-Z0-9_]+)\s+(\d+)u?\b", text)}
+    for body in re.findall(r"typedef enum \w*\s*\{(.*?)\}", text, flags=re.S):
+        body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+        consts.update({n: int(v) for n, v in re.findall(r"(FA_[A-Z_]+)\s*=\s*(\d+)", body)})
+    return consts
+
+
+def test_binding_constants_match_the_header(fa):
+    consts = _header_constants()
+    for name in ("FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_OOM",
+                 "FA_ERR_TIMEOUT", "FA_ERR_INTERNAL", "FA_MASK_CAUSAL", "FA_MASK_SLIDING_WINDOW",
+                 "FA_MASK_DOCUMENT", "FA_SCORE_NONE", "FA_SCORE_SOFTCAP", "FA_SCORE_ALIBI",
+                 "FA_DTYPE_F16", "FA_DTYPE_BF16"):
+        assert name in consts, name
+        assert getattr(fa, name) == consts[name], name
+
+
+def test_struct_layouts_match_the_header(fa):
+    # ctypes mirrors of the ABI structs: field order and sizes as declared (64-bit ABI).
+    assert ctypes.sizeof(fa.FaMaskParams) == 24      # int32, pad, void*, int32, pad
+    assert ctypes.sizeof(fa.FaScoreParams) == 16     # float, pad, const float*
+    assert ctypes.sizeof(fa.FaTensor) == 8 + 8 + 4 * 8 + 4 * 8
+    text = open(os.path.join(ROOT, "include", "fa_b200.h")).read()
+    for struct, fields in (("fa_mask_params", ["window", "doc_id", "separate_full_blocks"]),
+                           ("fa_score_params", ["softcap", "alibi_slopes"]),
+                           ("fa_tensor", ["data", "dtype", "B", "stride"])):
+        body = re.search(r"typedef struct %s \{(.*?)\}" % struct, text, flags=re.S).group(1)
+        body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+        pos = [body.index(f) for f in fields]
+        assert pos == sorted(pos), struct
