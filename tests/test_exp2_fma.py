@@ -57,3 +57,17 @@ def test_tiny_and_masked_inputs_stay_tiny_and_non_negative():
     a = np.array([-126.0, -127.0, -1000.0, -np.inf], dtype=np.float32)
     got = exp2_fma_model(a)
     assert np.all(got >= 0) and np.all(got < 2.0 ** -125)
+
+
+def test_coefficients_are_the_lawson_minimax_fit():
+    # The constants in the CUDA source are (to float32 precision of the fit) the minimax
+    # relative-error cubic that fit_exp2.py computes.
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_fit_exp2", os.path.join(ROOT, "block_sparse_masked_x128_b200", "fit_exp2.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    coeffs, rel = mod.fit()
+    src = np.array([float(c) for c in _coeffs()])
+    assert np.abs(src - coeffs).max() < 2e-6
+    assert rel < 7.6e-5
