@@ -466,8 +466,11 @@ def main(argv=None) -> int:
 
     if world > 1:
         import datetime
+        import torch
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        torch.cuda.set_device(local)   # one GPU per rank, bound before NCCL starts
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
     try:
         res = run_ours(args, w, world, rank, local)
     finally:
