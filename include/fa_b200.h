@@ -147,7 +147,8 @@ fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* par
  *   lse         device fp32 [B][H][Q_LEN] contiguous, or NULL to skip it
  *
  * Supported now: D in {64, 128}; Q_LEN and KV_LEN multiples of 128 (else
- * FA_ERR_UNSUPPORTED).  A query row with no allowed key gets out = 0, lse = -inf.
+ * FA_ERR_UNSUPPORTED).  q, k, v, out, lse and alibi_slopes must be memory of the current
+ * device (cudaMalloc or managed; host memory, pinned or not, gives FA_ERR_INVALID_ARG).  A query row with no allowed key gets out = 0, lse = -inf.
  * Device-side waits are bounded; a wait that runs out sets the mask's status word
  * (read it with fa_get_device_status) and the kernel returns early.
  */

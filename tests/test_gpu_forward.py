@@ -259,3 +259,29 @@ def test_long_sequence_sampled_rows(kind, window, score_kind):
     rows = _sample_rows(w.S, w.seed, n_random=6)
     O, L = run_oracle(w, q, k, v, rows=rows)
     compare(out, lse, O, L, rows=rows)
+
+
+def test_host_buffers_are_rejected_before_any_launch():
+    # The C ABI checks that every buffer is memory of the current device; host memory,
+    # pageable or pinned, is an argument error, and the context stays usable.
+    fa = fa_module()
+    g = torch.Generator().manual_seed(26)
+    q, k, v = (torch.randn(1, 2, 256, 64, generator=g).to(torch.bfloat16) for _ in range(3))
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    bm = gpu_block_mask(C, None, None, 256, 256)
+    for bad in (q, q.pin_memory()):
+        with pytest.raises(fa.FaError) as info:
+            fa.flex_attention(bad, kd, vd, bm)
+        assert info.value.status == fa.FA_ERR_INVALID_ARG
+    out_host = torch.empty(1, 2, 256, 64, dtype=torch.bfloat16).pin_memory()
+    with pytest.raises(fa.FaError):
+        fa.flex_attention(qd, kd, vd, bm, out=out_host)
+    lse_host = torch.empty(1, 2, 256, dtype=torch.float32).pin_memory()
+    with pytest.raises(fa.FaError):
+        fa.flex_attention(qd, kd, vd, bm, lse=lse_host)
+    out, lse = fa.flex_attention(qd, kd, vd, bm)
+    torch.cuda.synchronize()
+    assert bm.device_status() == fa.FA_OK
+    w = wl.Workload("host_check", B=1, H=2, S=256, D=64, dtype="bf16", mask_kind=C, seed=26)
+    O, L = run_oracle(w, q, k, v)
+    compare(out, lse, O, L)
