@@ -108,6 +108,9 @@ fa_status_t check_tensor(const fa_tensor_t* t, const char* name) {
     return FA_OK;
 }
 
+}  // namespace
+
+namespace fa {
 // Device memory of `dev` (cudaMalloc'd or managed); host and unregistered pointers are
 // rejected.  Leaves no CUDA error pending.
 fa_status_t check_device_memory(const void* ptr, int dev, const char* name) {
@@ -124,9 +127,6 @@ fa_status_t check_device_memory(const void* ptr, int dev, const char* name) {
     return FA_OK;
 }
 
-}  // namespace
-
-namespace fa {
 fa_status_t record_error(fa_status_t status, const char* message) {
     return fail(status, "%s", message);
 }
@@ -346,13 +346,13 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
     if (dev != m->device) return fail(FA_ERR_INVALID_ARG, "block_mask lives on device %d, current is %d", m->device, dev);
     // Every buffer the kernel touches must be memory of this device (a host pointer would
     // make the kernel fault instead of returning an error).
-    if ((s = check_device_memory(q->data, dev, "q")) != FA_OK) return s;
-    if ((s = check_device_memory(k->data, dev, "k")) != FA_OK) return s;
-    if ((s = check_device_memory(v->data, dev, "v")) != FA_OK) return s;
-    if ((s = check_device_memory(out->data, dev, "out")) != FA_OK) return s;
-    if (lse && (s = check_device_memory(lse, dev, "lse")) != FA_OK) return s;
+    if ((s = fa::check_device_memory(q->data, dev, "q")) != FA_OK) return s;
+    if ((s = fa::check_device_memory(k->data, dev, "k")) != FA_OK) return s;
+    if ((s = fa::check_device_memory(v->data, dev, "v")) != FA_OK) return s;
+    if ((s = fa::check_device_memory(out->data, dev, "out")) != FA_OK) return s;
+    if (lse && (s = fa::check_device_memory(lse, dev, "lse")) != FA_OK) return s;
     if (params && params->alibi_slopes &&
-        (s = check_device_memory(params->alibi_slopes, dev, "alibi_slopes")) != FA_OK)
+        (s = fa::check_device_memory(params->alibi_slopes, dev, "alibi_slopes")) != FA_OK)
         return s;
 
     CUtensorMap tq, tk, tv;

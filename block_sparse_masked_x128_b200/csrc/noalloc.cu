@@ -24,6 +24,11 @@ constexpr int kNoAllocMaxBlocks = 4096;  // query or kv blocks: Q_LEN, KV_LEN <=
 // Per-block document statistics of fa_create_block_mask_noalloc: 3 x 4096 int32 = 48 KiB.
 static __device__ __align__(256) int32_t g_doc_stats_scratch[3 * kNoAllocMaxBlocks];
 
+namespace fa {
+// Defined in api.cu: FA_OK when ptr is memory of device dev, else FA_ERR_INVALID_ARG.
+fa_status_t check_device_memory(const void* ptr, int dev, const char* name);
+}  // namespace fa
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -91,8 +96,18 @@ extern "C" fa_status_t fa_create_block_mask_noalloc(
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fa::record_error(FA_ERR_CUDA, "cudaGetDevice failed");
+    // The kernels write the four outputs and read doc_id directly: device memory only.
+    fa_status_t s;
+    if ((s = fa::check_device_memory(kv_num_blocks, dev, "kv_num_blocks")) != FA_OK ||
+        (s = fa::check_device_memory(kv_indices, dev, "kv_indices")) != FA_OK ||
+        (s = fa::check_device_memory(full_kv_num_blocks, dev, "full_kv_num_blocks")) != FA_OK ||
+        (s = fa::check_device_memory(full_kv_indices, dev, "full_kv_indices")) != FA_OK)
+        return s;
+    if ((mask_kind & FA_MASK_DOCUMENT) &&
+        (s = fa::check_device_memory(params->doc_id, dev, "doc_id")) != FA_OK)
+        return s;
     int32_t* scratch = nullptr;
-    const fa_status_t s = scratch_address(dev, &scratch);
+    s = scratch_address(dev, &scratch);
     if (s != FA_OK) return s;
 
     fa::MaskSpec spec;

@@ -174,7 +174,8 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
  *   kv_indices, full_kv_indices         int32 [B'][H'][q_blocks][kv_blocks]
  * with B' = max(B, 1), H' = max(H, 1), q_blocks = ceil(Q_LEN/128), kv_blocks =
  * ceil(KV_LEN/128); every element is written.  params->doc_id is read in place (not copied)
- * and must stay valid until the stream has run the build.
+ * and must stay valid until the stream has run the build.  The four buffers and doc_id must
+ * be memory of the current device (host memory gives FA_ERR_INVALID_ARG).
  *
  * Limit and scratch: Q_LEN and KV_LEN may not exceed 4096 blocks (524288 positions); larger
  * requests return FA_ERR_UNSUPPORTED.  Document statistics go to a fixed 48 KiB

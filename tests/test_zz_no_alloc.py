@@ -84,3 +84,14 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     st = fa._lib.fa_create_block_mask_noalloc(C, None, 0, 0, 128 * 4097, 128, 128, p, p, p, p, None)
     assert st == fa.FA_ERR_UNSUPPORTED
     assert "4096 blocks" in fa.fa_last_error_message()
+
+
+def test_noalloc_rejects_host_output_buffers():
+    fa = _fa()
+    dev = torch.zeros(4 * 4, dtype=torch.int32, device="cuda")
+    host = torch.zeros(4 * 4, dtype=torch.int32).pin_memory()
+    d, h = dev.data_ptr(), host.data_ptr()
+    st = fa._lib.fa_create_block_mask_noalloc(C, None, 0, 0, 512, 512, 128, h, d, d, d, None)
+    assert st == fa.FA_ERR_INVALID_ARG
+    assert "kv_num_blocks" in fa.fa_last_error_message()
+    torch.cuda.synchronize()
