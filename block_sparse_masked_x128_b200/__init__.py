@@ -287,15 +287,22 @@ def flex_attention(q, k, v, block_mask: BlockMask, *, score_mod: int = FA_SCORE_
         out = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty(q.shape[0], q.shape[1], q.shape[2], device=q.device, dtype=torch.float32)
+    if lse is not None:
+        # The C ABI takes lse as a bare pointer to [B][H][Q_LEN] fp32: check what it cannot.
+        if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous()
+                and tuple(lse.shape) == tuple(q.shape[:3]) and lse.device == q.device):
+            raise ValueError("lse must be a contiguous float32 CUDA tensor of shape (B, H, Q_LEN) "
+                             "on q's device")
     slopes_ptr = None
     if alibi_slopes is not None:
         if not (alibi_slopes.is_cuda and alibi_slopes.dtype == torch.float32):
             raise ValueError("alibi_slopes must be a float32 CUDA tensor")
         slopes_ptr = alibi_slopes.data_ptr()
     params = FaScoreParams(float(softcap), slopes_ptr)
-    fa_forward(fa_tensor(q), fa_tensor(k), fa_tensor(v), block_mask.handle, int(score_mod), params,
-               float(scale) if scale is not None else -1.0, fa_tensor(out),
-               lse.data_ptr() if lse is not None else None, stream)
+    with torch.cuda.device(q.device if q.is_cuda else block_mask.device):
+        fa_forward(fa_tensor(q), fa_tensor(k), fa_tensor(v), block_mask.handle, int(score_mod), params,
+                   float(scale) if scale is not None else -1.0, fa_tensor(out),
+                   lse.data_ptr() if lse is not None else None, stream)
     return out, lse
 
 

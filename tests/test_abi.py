@@ -159,3 +159,15 @@ def test_struct_layouts_match_the_header(fa):
         body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
         pos = [body.index(f) for f in fields]
         assert pos == sorted(pos), struct
+
+
+def test_binding_checks_lse_before_the_call(fa):
+    import torch
+
+    class _Mask:                      # never reached: the check comes first
+        handle, device = 0, None
+    q = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    for bad in (torch.zeros(1, 2, 128), torch.zeros(1, 2, 128, dtype=torch.float64),
+                torch.zeros(1, 2, 64)):
+        with pytest.raises(ValueError):
+            fa.flex_attention(q, q, q, _Mask(), lse=bad)

@@ -270,15 +270,24 @@ def test_host_buffers_are_rejected_before_any_launch():
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     bm = gpu_block_mask(C, None, None, 256, 256)
     for bad in (q, q.pin_memory()):
-        with pytest.raises(fa.FaError) as info:
+        with pytest.raises((fa.FaError, ValueError)):   # the binding or the C ABI refuses
             fa.flex_attention(bad, kd, vd, bm)
+        with pytest.raises(fa.FaError) as info:         # the C ABI on its own
+            fa.fa_forward(fa.fa_tensor(bad), fa.fa_tensor(kd), fa.fa_tensor(vd), bm.handle, 0,
+                          fa.FaScoreParams(30.0, None), -1.0, fa.fa_tensor(torch.empty_like(qd)),
+                          None, None)
         assert info.value.status == fa.FA_ERR_INVALID_ARG
     out_host = torch.empty(1, 2, 256, 64, dtype=torch.bfloat16).pin_memory()
     with pytest.raises(fa.FaError):
         fa.flex_attention(qd, kd, vd, bm, out=out_host)
     lse_host = torch.empty(1, 2, 256, dtype=torch.float32).pin_memory()
-    with pytest.raises(fa.FaError):
+    with pytest.raises(ValueError):          # the binding checks what a bare pointer cannot say
         fa.flex_attention(qd, kd, vd, bm, lse=lse_host)
+    with pytest.raises(fa.FaError) as info:  # and the C ABI rejects the host pointer itself
+        fa.fa_forward(fa.fa_tensor(qd), fa.fa_tensor(kd), fa.fa_tensor(vd), bm.handle, 0,
+                      fa.FaScoreParams(30.0, None), -1.0, fa.fa_tensor(torch.empty_like(qd)),
+                      lse_host.data_ptr(), None)
+    assert info.value.status == fa.FA_ERR_INVALID_ARG
     out, lse = fa.flex_attention(qd, kd, vd, bm)
     torch.cuda.synchronize()
     assert bm.device_status() == fa.FA_OK
