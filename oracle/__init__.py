@@ -1,8 +1,9 @@
 """Float64 CPU oracle for block-sparse masked attention.
 
 TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this package:
-only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may use it.  It shares no code with the CUDA library.
+only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU legs (the
+``cpu_baseline`` sample and the ``--impl reference`` arm) may use it.  It shares
+no code with the CUDA library.
 
 It is the plain definition of what the method computes, written out with
 materialised scores and an explicit dense mask, in the order and notation of
