@@ -82,11 +82,40 @@ def read_peaks() -> dict:
     return {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
 
 
+def _strip_c_comments(text: str) -> str:
+    """C/C++ source without comments, whitespace runs collapsed (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_sha() -> str:
+    """Hash of the forward kernel's code (comments and layout ignored), to tell whether the
+    recorded ncu counters still describe the kernel that runs."""
     h = hashlib.sha256()
-    for f in ("attn_fwd.cu", "fwd_common.cuh", "sm100_ptx.cuh", "fa_internal.h"):
-        with open(os.path.join(ROOT, "block_sparse_masked_x128_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    for rel in ("block_sparse_masked_x128_b200/csrc/attn_fwd.cu",
+                "block_sparse_masked_x128_b200/csrc/fwd_common.cuh",
+                "block_sparse_masked_x128_b200/csrc/sm100_ptx.cuh",
+                "block_sparse_masked_x128_b200/csrc/fa_internal.h", "include/fa_b200.h"):
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as fh:
+            h.update(_strip_c_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -121,3 +121,12 @@ def test_oracle_sample_rate_runs_at_least_one_chunk():
     q, k, v = wl.make_qkv(w)
     r = bench.oracle_sample_rate(w, q, k, v, None, 0.0, rows_per_chunk=8)
     assert r["rows"] == 8 and r["value"] > 0
+
+
+def test_kernel_hash_ignores_comments_and_layout():
+    a = 'int x = 1; // note\n/* block\n comment */ asm volatile("ld.x // not a comment");\n'
+    b = 'int  x = 1;\n\nasm volatile("ld.x // not a comment"); // other words\n'
+    assert bench._strip_c_comments(a) == bench._strip_c_comments(b)
+    assert "not a comment" in bench._strip_c_comments(a)
+    assert bench._strip_c_comments("int x = 1;") != bench._strip_c_comments("int x = 2;")
+    assert len(bench.kernel_source_sha()) == 16
