@@ -7,23 +7,30 @@
 // tiles and never writing the score matrix to memory.
 //
 // Organisation (one persistent CTA per SM, 12 warps):
-//   warp 0      TMA producer: Q tiles of the unit, then K_j, V_j of every listed kv block
-//               into a ring of shared-memory stages (128-byte swizzle).
+//   warp 0      TMA producer (fwd_common.cuh): takes the next unit from the global counter,
+//               publishes it to the other roles through a shared-memory ring, then loads
+//               the unit's Q tiles and K_j, V_j of every listed kv block into a ring of
+//               shared-memory stages (128-byte swizzle).
 //   warp 1      MMA issuer (one elected lane): S_t = Q_t K_j^T into TMEM (SS MMA), and
 //               O_t += P_t V_j with P_t read from TMEM (TS MMA).
-//   warps 2-3   TMEM allocation / release only.
+//   warp 2      TMEM allocation / release; warp 3 idle (completes the warpgroup).
 //   warps 4-7   softmax for query tile 0 (one thread per query row = TMEM lane),
 //   warps 8-11  softmax for query tile 1.
 // A work unit is a pair of adjacent query blocks (2p, 2p+1) of one (b, h); both tiles
-// share every K/V load of the merged kv-block list and ping-pong on the tensor core:
-// while one softmax group works on its S tile, the MMA warp feeds the other.
+// share every K/V load of the merged kv-block list.  The MMA warp serves tile 0, then
+// tile 1, for every entry; that fixed order keeps the two softmax groups about half a
+// tile apart, so one group's exponentials run while the other waits for its next S.
 //
-// TMEM (512 columns x 128 lanes, fp32): S0 at column 0, S1 at 128, O0 at 256, O1 at
-// 256 + D.  P_t (16-bit, two per column) overwrites the first 64 columns of S_t.
+// TMEM (512 columns x 128 lanes, fp32):
+//   D = 64:  S0 at 0, S1 at 128, P0 at 256, P1 at 320 (16-bit pairs), O0 at 384, O1 at 448;
+//            the next S_t may be computed while P_t is still being written (S_free).
+//   D = 128: S0 at 0, S1 at 128, O0 at 256, O1 at 384; P_t overwrites the first 64
+//            columns of S_t, so P.V of an entry is issued before the next S_t.
 //
 // Softmax: running max in log2 units with a lazy rescale -- O and the row sum are
 // rescaled only when the max grows by more than 8 (a factor 256), which keeps P <= 256
-// and is exact because the final division uses the same stale max.  All waits are
+// and is exact because the final division uses the same stale max.  The score_mod kind
+// and the presence of a document predicate are template parameters.  All waits are
 // bounded; a wait that runs out sets the status word and every role unwinds.
 #include <cfloat>
 
@@ -313,7 +320,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
     uint32_t u_iter = 0;
     bool taken = true;
     // The next unit is taken before this unit's epilogue waits for O, so the ring handshake
-    // and the schedule reads overlap the last P.V instead of following it.
+    // overlaps the last P.V instead of following it.
     int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, taken);
     for (;;) {
         if (u < 0) return;
