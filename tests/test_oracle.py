@@ -344,6 +344,11 @@ def test_document_lengths_of_the_packed_workload():
     assert ids.shape == (8192,) and ids.dtype == np.int32
     assert np.array_equal(np.unique(ids), np.arange(4))
     assert np.all(np.diff(ids) >= 0)
+    # The stated recipe: three sorted cuts from default_rng(4).integers(0, 6145, 3), the gaps
+    # of [0, cuts, 6144], each plus 512.
+    cuts = np.sort(np.random.default_rng(4).integers(0, 6145, 3))
+    edges = np.concatenate([[0], cuts, [6144]])
+    assert list(lens) == [int(g) + 512 for g in np.diff(edges)] == [4975, 1465, 891, 861]
 
 
 def test_three_document_example_of_the_page():
