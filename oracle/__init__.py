@@ -18,8 +18,8 @@ the pages (see each function's docstring for the passage it follows):
                                                 the backward pass, not built yet)
 
 Every function is pinned by a "not gpu" test against facts the pages or the
-mathematics fix; the one reading with no such pin (the composition order of
-soft-cap and ALiBi) is marked "parity unpinned" where it is defined.
+mathematics fix; where a function follows a reading of the pages (the composition
+order of soft-cap and ALiBi, for one), the pin checks that reading.
 """
 from .backward import attention_backward, make_score_mod_grad, soft_cap_grad  # noqa: F401
 from .attention import (  # noqa: F401

@@ -133,9 +133,11 @@ def alibi(slopes):
 def compose_score_mods(*mods):
     """Apply score_mods left to right.
 
-    Parity unpinned: with both soft-cap and ALiBi, the pages fix no order.
-    Reading: soft-cap first, then the bias (30*tanh(s/30) + bias), so the
-    distance penalty is not squashed into [-30, 30].
+    With both soft-cap and ALiBi the pages fix no order.  Reading: soft-cap first, then
+    the bias (30*tanh(s/30) + bias), so the distance penalty is not squashed into
+    [-30, 30].  The composition is pinned to that reading by closed forms: scores
+    s = cap*ln(a), whose capped value is the rational cap*(a^2-1)/(a^2+1), plus the
+    exact bias -2^-(h+1)*(q_idx - kv_idx).
     """
     def score_mod(score, b, h, q_idx, kv_idx):
         for m in mods:

@@ -7,6 +7,7 @@ the oracle's inputs or functors and checks that a pin catches each one.
 """
 import math
 import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -320,6 +321,59 @@ def test_alibi_matches_a_hand_written_bias_matrix():
     qi, ki = np.arange(4)[:, None], np.arange(4)[None, :]
     for h in (0, 1):
         assert np.array_equal(sm(np.zeros((4, 4)), 0, h, qi, ki), np.array(bias[h]))
+
+
+# Soft-cap then ALiBi ("Bonus: a score_mod for soft-capping" for the cap; the bias is the
+# additive distance penalty of "The two hooks"; the order is the stated reading: cap first,
+# then add slope_h * (kv_idx - q_idx)).  Scores are chosen as s = cap * ln(a), where
+# tanh(ln a) = (a^2 - 1) / (a^2 + 1) exactly, so every expected value is a rational closed
+# form computed here without a tanh; the H = 8 slopes are 2^-(h+1).
+_COMPOSE_A = [Fraction(1), Fraction(2), Fraction(3), Fraction(1, 3), Fraction(1, 10), Fraction(1000)]
+_COMPOSE_H = [0, 3, 7]
+_COMPOSE_DIST = [0, 1, 37, 16383]          # q_idx - kv_idx >= 0: keys a causal mask keeps
+
+
+def _compose_table(cap=30):
+    rows = []
+    for a in _COMPOSE_A:
+        capped = Fraction(cap) * (a * a - 1) / (a * a + 1)
+        for h in _COMPOSE_H:
+            for d in _COMPOSE_DIST:
+                rows.append((cap * math.log(float(a)), h, d,
+                             float(capped - Fraction(d, 2 ** (h + 1)))))
+    return rows
+
+
+def _apply(sm, s, h, d):
+    q_idx = np.array([[d + 5]])
+    kv_idx = np.array([[5]])
+    return float(sm(np.array([[s]]), 0, h, q_idx, kv_idx)[0, 0])
+
+
+def test_soft_cap_then_alibi_matches_closed_forms():
+    sm = oracle.make_score_mod(oracle.SCORE_SOFTCAP | oracle.SCORE_ALIBI, H=8, softcap=30.0)
+    for s, h, d, want in _compose_table():
+        got = _apply(sm, s, h, d)
+        assert abs(got - want) <= 1e-12 * max(1.0, abs(want)), (s, h, d, got, want)
+
+
+def test_composition_pin_catches_the_bias_inside_the_tanh():
+    slopes = oracle.alibi_slopes(8)
+    wrong = lambda s, b, h, qi, ki: 30.0 * np.tanh((s + slopes[h] * (ki - qi)) / 30.0)
+    bad = [abs(_apply(wrong, s, h, d) - want) > 1e-6 for s, h, d, want in _compose_table()]
+    assert any(bad) and sum(bad) >= len(bad) // 2
+
+
+def test_composition_pin_catches_the_cap_applied_after_the_bias():
+    wrong = oracle.compose_score_mods(oracle.alibi(oracle.alibi_slopes(8)), oracle.soft_cap(30.0))
+    bad = [abs(_apply(wrong, s, h, d) - want) > 1e-6 for s, h, d, want in _compose_table()]
+    assert any(bad) and sum(bad) >= len(bad) // 2
+
+
+def test_composition_pin_catches_a_slope_of_the_wrong_head():
+    shifted = np.concatenate([[1.0], oracle.alibi_slopes(8)[:-1]])    # 2^-h instead of 2^-(h+1)
+    wrong = oracle.compose_score_mods(oracle.soft_cap(30.0), oracle.alibi(shifted))
+    assert any(abs(_apply(wrong, s, h, d) - want) > 1e-6 for s, h, d, want in _compose_table())
 
 
 def test_score_mod_only_changes_live_values():
