@@ -12,7 +12,6 @@ FlexAttention API the pages use ("How to Use FlexAttention on Apple Silicon", Se
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 from typing import Optional, Tuple
 
@@ -259,6 +258,19 @@ class BlockMask:
                 pass
 
 
+def check_doc_id(doc_id, KV_LEN: int, device) -> None:
+    """Raise ValueError unless doc_id is a contiguous 1-D int32 tensor of KV_LEN ids on
+    `device` (the library reads exactly KV_LEN ids through a bare pointer)."""
+    import torch
+    if not (doc_id.is_cuda and doc_id.dtype == torch.int32 and doc_id.is_contiguous()):
+        raise ValueError("doc_id must be a contiguous int32 CUDA tensor")
+    if doc_id.dim() != 1 or doc_id.numel() != int(KV_LEN):
+        raise ValueError(f"doc_id must hold exactly KV_LEN={int(KV_LEN)} ids, got shape "
+                         f"{tuple(doc_id.shape)}")
+    if doc_id.device != torch.device(device):
+        raise ValueError(f"doc_id lives on {doc_id.device}, the mask on {device}")
+
+
 def create_block_mask(mask_kind: int, B: Optional[int], H: Optional[int], Q_LEN: int, KV_LEN: int,
                       *, window: int = 0, doc_id=None, separate_full_blocks: bool = True,
                       BLOCK_SIZE: int = 128, device=None, stream=None) -> BlockMask:
@@ -267,8 +279,8 @@ def create_block_mask(mask_kind: int, B: Optional[int], H: Optional[int], Q_LEN:
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     doc_ptr = None
     if doc_id is not None:
-        if not (doc_id.is_cuda and doc_id.dtype == torch.int32 and doc_id.is_contiguous()):
-            raise ValueError("doc_id must be a contiguous int32 CUDA tensor")
+        # The C ABI reads KV_LEN ids through a bare pointer: check what it cannot.
+        check_doc_id(doc_id, KV_LEN, dev)
         doc_ptr = doc_id.data_ptr()
     params = FaMaskParams(int(window), doc_ptr, 1 if separate_full_blocks else 0)
     with torch.cuda.device(dev):
@@ -295,8 +307,12 @@ def flex_attention(q, k, v, block_mask: BlockMask, *, score_mod: int = FA_SCORE_
                              "on q's device")
     slopes_ptr = None
     if alibi_slopes is not None:
-        if not (alibi_slopes.is_cuda and alibi_slopes.dtype == torch.float32):
-            raise ValueError("alibi_slopes must be a float32 CUDA tensor")
+        # The kernel reads slope h for h < H through a bare pointer: H contiguous floats.
+        if not (alibi_slopes.is_cuda and alibi_slopes.dtype == torch.float32
+                and alibi_slopes.is_contiguous() and alibi_slopes.numel() == q.shape[1]
+                and alibi_slopes.device == q.device):
+            raise ValueError("alibi_slopes must be a contiguous float32 CUDA tensor of H "
+                             "values on q's device")
         slopes_ptr = alibi_slopes.data_ptr()
     params = FaScoreParams(float(softcap), slopes_ptr)
     with torch.cuda.device(q.device if q.is_cuda else block_mask.device):
@@ -305,6 +321,3 @@ def flex_attention(q, k, v, block_mask: BlockMask, *, score_mod: int = FA_SCORE_
                    lse.data_ptr() if lse is not None else None, stream)
     return out, lse
 
-
-def default_scale(D: int) -> float:
-    return 1.0 / math.sqrt(D)

@@ -11,7 +11,9 @@
 //
 // The array is a file-scope __device__ variable, so every GPU that loads this library
 // holds it (48 KiB) until the process exits.  Host code cannot use its name as a device
-// address; the address is fetched once per device with cudaGetSymbolAddress.  All calls
+// address; the address is fetched once per device with cudaGetSymbolAddress and kept for
+// the life of the process, so the entry point must not be used across a cudaDeviceReset
+// (the module is reloaded then and the array may move).  All calls
 // share the array and it keeps the last call's contents; every entry a call reads is
 // written earlier by the same call, so nothing has to start at zero.  Two calls whose
 // work overlaps on the GPU (for example on two streams) race on the array.

@@ -25,9 +25,13 @@
  *     argument checks happen before any launch; on an error nothing is launched and
  *     no output is written.  fa_last_error_message() gives a one-line reason.
  *   - Library objects are not thread-safe against concurrent destroy; concurrent
- *     fa_forward calls on one mask from different streams are allowed, up to 64 in
- *     flight at once (the lists are read-only for them; each launch takes the next of
- *     the mask's 64 pairs of work-distribution counters, which its kernel leaves zero).
+ *     fa_forward calls on one mask, from any threads and streams, are allowed (the lists
+ *     are read-only for them).  Each launch takes the next of the mask's 64 pairs of
+ *     work-distribution counters, which its kernel leaves zero; before a pair is reused the
+ *     new launch's stream waits on the GPU for the previous user of that pair, so a 65th
+ *     forward in flight is delayed, never corrupted.  Under stream capture that wait is not
+ *     recorded: a captured forward keeps its pair for every replay, and replays must not
+ *     overlap other forwards on the same mask.
  */
 #ifndef FA_B200_H
 #define FA_B200_H
@@ -77,7 +81,8 @@ typedef struct fa_mask_params {
 
 typedef struct fa_score_params {
     float        softcap;        /* > 0 when FA_SCORE_SOFTCAP is set (30 in the soft-capping example) */
-    const float* alibi_slopes;   /* device [H] fp32, or NULL for the slopes 2^(-8(h+1)/H)              */
+    const float* alibi_slopes;   /* device, H contiguous fp32 slopes (slope h at index h), or NULL for
+                                    the slopes 2^(-8(h+1)/H)                                           */
 } fa_score_params_t;
 
 /* A (B, H, S, D) tensor: batch, heads, sequence, head_dim, the layout shared with
@@ -182,8 +187,9 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
  * __device__ array that every GPU loading this library holds until exit.  All calls share
  * it (it keeps the last call's contents; each call writes every entry it reads), so calls
  * whose work overlaps on the GPU -- e.g. on two streams -- race.  The first call on a
- * device looks up the array's address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture.
+ * device looks up the array's address (cudaGetSymbolAddress) with that device current and
+ * keeps it for the life of the process; make that first call before any stream capture, and
+ * do not use this entry point across a cudaDeviceReset of that device.
  */
 fa_status_t fa_create_block_mask_noalloc(uint32_t mask_kind, const fa_mask_params_t* params,
                                          int32_t B, int32_t H, int32_t Q_LEN, int32_t KV_LEN,

@@ -171,3 +171,37 @@ def test_binding_checks_lse_before_the_call(fa):
                 torch.zeros(1, 2, 64)):
         with pytest.raises(ValueError):
             fa.flex_attention(q, q, q, _Mask(), lse=bad)
+
+
+class _FakeCudaIds:
+    """Stands in for a CUDA int32 tensor (no GPU here): only what check_doc_id reads."""
+
+    def __init__(self, n, device="cuda:0", dims=1):
+        import torch
+        self.is_cuda = True
+        self.dtype = torch.int32
+        self.device = torch.device(device)
+        self.shape = (n,) if dims == 1 else (1, n)
+        self._n = n
+        self._dims = dims
+
+    def is_contiguous(self):
+        return True
+
+    def dim(self):
+        return self._dims
+
+    def numel(self):
+        return self._n
+
+
+def test_binding_rejects_a_doc_id_shorter_than_kv_len(fa):
+    # The C ABI reads KV_LEN ids through a bare pointer; a short vector would be read out of
+    # bounds on the device, so the binding refuses it before anything is launched.
+    with pytest.raises(ValueError, match="KV_LEN=1024"):
+        fa.check_doc_id(_FakeCudaIds(1000), 1024, "cuda:0")
+    with pytest.raises(ValueError, match="KV_LEN"):
+        fa.check_doc_id(_FakeCudaIds(1024, dims=2), 1024, "cuda:0")
+    with pytest.raises(ValueError, match="lives on"):
+        fa.check_doc_id(_FakeCudaIds(1024, device="cuda:1"), 1024, "cuda:0")
+    fa.check_doc_id(_FakeCudaIds(1024), 1024, "cuda:0")
