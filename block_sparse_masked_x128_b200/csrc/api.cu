@@ -108,6 +108,43 @@ fa_status_t check_tensor(const fa_tensor_t* t, const char* name) {
     return FA_OK;
 }
 
+// Launch a forward-type kernel with a pair of unit counters of its own (the kernel's last CTA
+// returns them to zero, also after a timeout).  The pairs are taken round robin; before a pair
+// is reused, the stream waits (on the GPU) for the event recorded after its previous user, so
+// however many forwards are enqueued on one mask, at most kSchedCtrSlots share the pairs at
+// once and none ever shares a pair with another that is still running.  Under stream capture
+// no event is recorded or waited on: a captured forward keeps the pair it was given for every
+// replay, and the caller orders replays against other work on the same mask.
+template <class Launch>
+fa_status_t launch_with_counter_pair(fa_block_mask_t* m, cudaStream_t st, Launch&& launch) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(st, &cap);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    const bool capturing = cap != cudaStreamCaptureStatusNone;
+    std::lock_guard<std::mutex> lock(m->ctr_mutex);
+    const uint32_t slot = m->next_ctr++ % fa::kSchedCtrSlots;
+    cudaEvent_t& ev = m->ctr_event[slot];
+    if (!capturing) {
+        if (ev) {
+            e = cudaStreamWaitEvent(st, ev, 0);
+            if (e != cudaSuccess) return cuda_fail(e, "waiting for the previous user of a counter pair");
+        } else {
+            e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+            if (e != cudaSuccess) {
+                ev = nullptr;
+                return cuda_fail(e, "cudaEventCreateWithFlags");
+            }
+        }
+    }
+    e = launch(m->sched_ctr + 2 * slot);
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    if (!capturing) {
+        e = cudaEventRecord(ev, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord after the forward");
+    }
+    return ok();
+}
+
 }  // namespace
 
 namespace fa {
@@ -281,6 +318,8 @@ void fa_destroy_block_mask(fa_block_mask_t* m) {
     int cur = 0;
     cudaGetDevice(&cur);
     if (cur != m->device) cudaSetDevice(m->device);
+    for (cudaEvent_t ev : m->ctr_event)
+        if (ev) cudaEventDestroy(ev);
     cudaFree(m->dev_base);
     if (cur != m->device) cudaSetDevice(cur);
     delete m;
@@ -393,22 +432,17 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
     p.out_stride[2] = out->stride[2];
     p.lse = lse;
     p.status = m->status;
-    {
-        // A pair of unit counters of its own for this launch (the kernel's last CTA returns
-        // them to zero, also after a timeout).
-        fa_block_mask_t* mm = const_cast<fa_block_mask_t*>(m);
-        const uint32_t slot = mm->next_ctr.fetch_add(1, std::memory_order_relaxed) % fa::kSchedCtrSlots;
-        p.sched_ctr = m->sched_ctr + 2 * slot;
-    }
     p.stall_loads = g_stall_loads.load(std::memory_order_relaxed);
 
     const int nsm = sm_count(dev);
     if (nsm <= 0) return fail(FA_ERR_CUDA, "could not read the SM count");
     const int grid = p.n_units < nsm ? p.n_units : nsm;
-    e = fa::launch_attn_fwd(p, (int)q->D, q->dtype == FA_DTYPE_BF16, (int)score_mod_kind, tq, tk, tv,
-                            grid, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
-    return ok();
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return launch_with_counter_pair(const_cast<fa_block_mask_t*>(m), st, [&](int32_t* ctr) {
+        p.sched_ctr = ctr;
+        return fa::launch_attn_fwd(p, (int)q->D, q->dtype == FA_DTYPE_BF16, (int)score_mod_kind,
+                                   tq, tk, tv, grid, st);
+    });
 }
 
 // Test hook for failure detection (see the header): read by every later fa_forward.

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <atomic>
+#include <mutex>
 
 #include <cstddef>
 #include <cstdint>
@@ -105,5 +106,10 @@ struct fa_block_mask {
     int32_t* sched_order;
     int32_t* status;
     int32_t* sched_ctr;       // fa::kSchedCtrSlots pairs of unit counters after the status word
-    std::atomic<uint32_t> next_ctr{0};  // round-robin pick of a counter pair per forward
+    // Round-robin pick of a counter pair per forward.  ctr_event[s] is recorded after the
+    // last forward that used pair s; the next forward on pair s waits for it on the GPU, so
+    // no more than kSchedCtrSlots forwards ever share the pairs at once.
+    std::mutex ctr_mutex;
+    uint32_t next_ctr = 0;
+    cudaEvent_t ctr_event[fa::kSchedCtrSlots] = {};
 };

@@ -248,6 +248,34 @@ def test_many_forwards_reuse_the_counters():
     assert bm.device_status() == fa.FA_OK
 
 
+def test_more_forwards_in_flight_than_counter_pairs():
+    # Four streams are held back by a sleep kernel while 160 forwards are enqueued on one mask:
+    # more than its 64 counter pairs are pending at once.  A forward that would reuse a pair
+    # waits on the GPU for the pair's previous user, so every output is still exact.
+    fa = fa_module()
+    g = torch.Generator().manual_seed(27)
+    q, k, v = (torch.randn(1, 4, 1024, 64, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    bm = gpu_block_mask(C, None, None, 1024, 1024)
+    o_ref, l_ref = fa.flex_attention(q, k, v, bm)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    outs = []
+    for st in streams:
+        with torch.cuda.stream(st):
+            torch.cuda._sleep(20_000_000)          # about 10 ms: the launches below queue up
+    for i in range(160):
+        st = streams[i % 4]
+        with torch.cuda.stream(st):
+            out = torch.empty_like(q)
+            lse = torch.empty(1, 4, 1024, device="cuda")
+            fa.flex_attention(q, k, v, bm, out=out, lse=lse, stream=st)
+            outs.append((out, lse))
+    torch.cuda.synchronize()
+    assert bm.device_status() == fa.FA_OK
+    for out, lse in outs:
+        assert torch.equal(out, o_ref) and torch.equal(lse, l_ref)
+
+
 @pytest.mark.parametrize("kind,window,score_kind", [(C, 0, wl.SCORE_NONE),
                                                     (C | SW, 4096, wl.SCORE_SOFTCAP | wl.SCORE_ALIBI)])
 def test_long_sequence_sampled_rows(kind, window, score_kind):
