@@ -20,7 +20,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -133,59 +132,78 @@ def recorded_traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock, power and clock-event reasons sampled through NVML while the timed region runs.
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Only reads: nothing here changes a GPU setting.  A thread polls every `period_s`; entering
+    the context waits for the first sample, so even a region of a few milliseconds holds
+    samples taken while its kernels run.
+    """
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index: int, period_s: float = 0.0005):
+        self.cuda_index = cuda_index
+        self.period = period_s
+        self.samples = []          # (sm_mhz, power_w, reasons bitmask)
+        self.sm_max = None
+        self.error = None
+        self._stop = threading.Event()
+        self._first = threading.Event()
+        self._thread = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
+
+    def _run(self):
+        try:
+            import pynvml
+            h = self._handle()
+            self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            while True:
+                sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))
+                self.samples.append((sm, pw, rs))
+                self._first.set()
+                if self._stop.wait(self.period):
+                    break
+        except Exception as exc:   # no NVML: the summary says so
+            self.error = f"{type(exc).__name__}: {exc}"
+        finally:
+            self._first.set()
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.reader = threading.Thread(target=self._read, daemon=True)
-            self.reader.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        self._first.wait(timeout=10)
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.reader.join(timeout=2)
+        self._stop.set()
+        self._thread.join(timeout=10)
 
     def summary(self) -> dict:
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [x[0] for x in self.samples]
+        reasons = set()
+        for _, _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.sm_max,
+               "sm_mhz_min": min(sm) if sm else None,
+               "power_w_max": max(x[1] for x in self.samples) if sm else None,
+               "reasons": sorted(reasons), "samples": len(sm), "source": "nvml"}
+        if self.error:
+            out["error"] = self.error
+        return out
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -269,6 +287,13 @@ def cores_used() -> int:
 
 # ---------------------------------------------------------------- arms
 
+def rank_plan(w: wl.Workload, world: int, rank: int) -> dict:
+    """What rank `rank` of `world` runs: its own batch of the workload (data parallel, weak
+    scaling), drawn from its own seed, with no exchange on the data path."""
+    return {"seed": w.seed + 1000 * rank, "global_batch": w.B * world,
+            "parallelism": f"dp{world}"}
+
+
 def config_dict(w: wl.Workload, world: int) -> dict:
     mask = []
     if w.mask_kind & wl.MASK_CAUSAL:
@@ -282,27 +307,27 @@ def config_dict(w: wl.Workload, world: int) -> dict:
         score.append(f"softcap({w.softcap:g})")
     if w.score_kind & wl.SCORE_ALIBI:
         score.append("alibi(2^(-8(h+1)/H))")
+    plan = rank_plan(w, world, 0)
     return {"workload": w.name, "B": w.B, "H": w.H, "Q_LEN": w.S, "KV_LEN": w.S, "head_dim": w.D,
             "BLOCK_SIZE": 128, "mask_mod": " & ".join(mask) or "none",
-            "score_mod": " then ".join(score) or "none", "global_batch": w.B * world,
-            "seq_len": w.S, "parallelism": f"dp{world}",
+            "score_mod": " then ".join(score) or "none", "global_batch": plan["global_batch"],
+            "seq_len": w.S, "parallelism": plan["parallelism"],
             "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write) before every timed step"}
 
 
-def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
+def time_forward(w: wl.Workload, steps: int, warmup: int, world: int, rank: int, dev) -> dict:
+    """Build the mask (timed apart), then time `steps` forwards with CUDA events on the
+    launching stream, L2 flushed before each, clocks sampled during the timed region."""
     import torch
     import block_sparse_masked_x128_b200 as fa
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    q, k, v = wl.make_qkv(w, seed=w.seed + 1000 * rank)
+    q, k, v = wl.make_qkv(w, seed=rank_plan(w, world, rank)["seed"])
     doc = wl.make_doc_ids(w)
     flops = flops_per_step(w, doc)
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
     doc_d = torch.from_numpy(doc).to(dev) if doc is not None else None
     stream = torch.cuda.current_stream()
 
-    # Mask build (once per shape; timed apart from the forward).
     build_ms = []
     bm = None
     for _ in range(5):
@@ -320,20 +345,20 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
         fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap or 30.0,
                           scale=w.scale, out=out, lse=lse)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
         fwd()
     torch.cuda.synchronize()
     if bm.device_status() != fa.FA_OK:
         raise RuntimeError("a device-side wait timed out during warm-up")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
+    with ClockSampler(dev.index) as clocks:
         t_wall0 = time.perf_counter()
-        for i in range(args.steps):
+        for i in range(steps):
             flush.zero_()
             starts[i].record(stream)
             fwd()
@@ -344,10 +369,26 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
     if bm.device_status() != fa.FA_OK:
         raise RuntimeError("a device-side wait timed out during the timed steps")
     per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    t_fwd_ms = sum(per)
-    t_max_ms = max_over_ranks(t_fwd_ms, world, dev)
-    value = world * flops * args.steps / (t_max_ms * 1e-3) / 1e12
-    achieved = flops / (statistics.mean(per) * 1e-3) / 1e12
+    t_max_ms = max_over_ranks(sum(per), world, dev)
+    ck = clocks.summary()
+    return {"flops": flops, "per_ms": per, "t_max_ms": t_max_ms,
+            "value": world * flops * steps / (t_max_ms * 1e-3) / 1e12,
+            "achieved": flops / (statistics.mean(per) * 1e-3) / 1e12,
+            "mask_build_ms": statistics.median(build_ms[1:]), "clocks": ck, "wall_s": t_wall,
+            "q": q, "k": k, "v": v, "doc": doc, "qd": qd, "kd": kd, "vd": vd, "out": out,
+            "lse": lse, "bm": bm}
+
+
+def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
+    import torch
+    import block_sparse_masked_x128_b200 as fa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = read_peaks()
+    tf = time_forward(w, args.steps, args.warmup, world, rank, dev)
+    flops, out, lse, bm = tf["flops"], tf["out"], tf["lse"], tf["bm"]
+    stream = torch.cuda.current_stream()
 
     # End to end through the public API from pinned host buffers: every step copies its q, k,
     # v in, runs the forward and copies out and lse back.  Two device buffer sets and three
@@ -355,6 +396,8 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
     # and step i-1's output copy, as a user streaming batches would run it.
     e2e = None
     if not args.no_e2e:
+        q, k, v = tf["q"], tf["k"], tf["v"]
+        qd, kd, vd = tf["qd"], tf["kd"], tf["vd"]
         qh, kh, vh = (t.pin_memory() for t in (q, k, v))
         e2e_steps = max(3, min(args.steps, args.e2e_steps))
         s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
@@ -408,28 +451,54 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
                "d2h_bytes_per_step": int(out.numel() * out.element_size() + lse.numel() * 4),
                "steps": e2e_steps, "pipelined": "copy-in / forward / copy-out on three streams"}
 
-    peaks = read_peaks()
     traffic = recorded_traffic(w.name)
+    ck = tf["clocks"]
+    ms_step = tf["t_max_ms"] / args.steps
     res = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": t_max_ms / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": tf["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": config_dict(w, world),
-        "pct_of_peak": 100.0 * value / world / peaks["bf16_tflops"],
-        "pct_of_nominal_2250": 100.0 * value / world / NOMINAL_BF16_TFLOPS,
+        "pct_of_peak": 100.0 * tf["value"] / world / peaks["bf16_tflops"],
+        "pct_of_nominal_2250": 100.0 * tf["value"] / world / NOMINAL_BF16_TFLOPS,
         "live_gflop_per_step": flops / 1e9,
-        "mask_build_ms": statistics.median(build_ms[1:]),
+        "mask_build_ms": tf["mask_build_ms"],
         "gpu_launches": args.steps,
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+        "roofline": {"bound": "tensor", "achieved": tf["achieved"], "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": tf["achieved"] / peaks["bf16_tflops"],
                      "traffic": traffic, "peak_source": peaks["source"] + " bf16_tflops (burst)",
                      "kernel": "attn_fwd_kernel"},
-        "clocks": clocks.summary(),
-        "wall_s_timed_region": t_wall,
+        "clocks": ck,
+        "ms_x_sm_mhz": ms_step * ck["sm_mhz"] if ck.get("sm_mhz") else None,
+        "wall_s_timed_region": tf["wall_s"],
     }
     if e2e is not None:
         res["e2e"] = e2e
+    del tf
+
+    # The other workloads, measured the same way in the same process (the 32k soft-cap + ALiBi
+    # one is the second headline configuration).
+    if not args.no_per_workload:
+        per = {}
+        for other in wl.WORKLOADS:
+            if other.name == w.name:
+                continue
+            o = time_forward(other, args.steps, args.warmup, world, rank, dev)
+            oms = o["t_max_ms"] / args.steps
+            per[other.name] = {
+                "value": o["value"], "unit": UNIT, "ms_per_step": oms,
+                "frac": o["achieved"] / peaks["bf16_tflops"],
+                "live_gflop_per_step": o["flops"] / 1e9, "mask_build_ms": o["mask_build_ms"],
+                "traffic": recorded_traffic(other.name), "clocks": o["clocks"],
+                "ms_x_sm_mhz": oms * o["clocks"]["sm_mhz"] if o["clocks"].get("sm_mhz") else None,
+                "gpu_launches": args.steps}
+            del o
+            torch.cuda.empty_cache()
+        res["per_workload"] = per
+
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        q, k, v = wl.make_qkv(w, seed=rank_plan(w, world, rank)["seed"])
+        doc = wl.make_doc_ids(w)
         cb = oracle_sample_rate(w, q, k, v, doc, args.cpu_seconds)
         res["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cores_used(),
                                "kind": "oracle",
@@ -477,6 +546,8 @@ def main(argv=None) -> int:
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="time only --workload (skip the per_workload section)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-budget-s", type=float, default=60.0)
     args = ap.parse_args(argv)

@@ -41,20 +41,30 @@ def _free_port():
 
 
 def _rank_main(rank, world, port, out):
+    import torch
     import torch.distributed as dist
     os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port),
                        "RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank)})
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         assert bench.dist_env() == (world, rank, rank)
+        # The per-rank partition bench.py runs: each rank draws its own batch from its own seed.
+        w = wl.WORKLOADS[1].scaled(S=256, H=2)
+        plan = bench.rank_plan(w, world, rank)
+        q, k, v = wl.make_qkv(w, seed=plan["seed"])
+        sums = torch.tensor([float(q.float().sum()), float(plan["seed"])], dtype=torch.float64)
+        gathered = [torch.zeros(2, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(gathered, sums)
+        cfg = bench.config_dict(w, world)
         t = bench.max_over_ranks(10.0 + 5.0 * rank, world)
         bench.barrier(world)
-        out[rank] = t
+        out[rank] = {"t": t, "plan": plan, "cfg": (cfg["global_batch"], cfg["parallelism"]),
+                     "gathered": [g.tolist() for g in gathered]}
     finally:
         dist.destroy_process_group()
 
 
-def test_max_over_ranks_with_two_gloo_ranks():
+def test_two_gloo_ranks_partition_the_work_and_take_the_max_time():
     ctx = mp.get_context("spawn")
     out = ctx.Manager().dict()
     port = _free_port()
@@ -64,7 +74,15 @@ def test_max_over_ranks_with_two_gloo_ranks():
     for p in procs:
         p.join(120)
         assert p.exitcode == 0
-    assert out[0] == out[1] == 15.0
+    r0, r1 = out[0], out[1]
+    assert r0["t"] == r1["t"] == 15.0                     # max over ranks, on every rank
+    assert r0["plan"]["seed"] != r1["plan"]["seed"]       # independent batches
+    assert r0["plan"]["seed"] == wl.WORKLOADS[1].seed and r1["plan"]["seed"] == wl.WORKLOADS[1].seed + 1000
+    assert r0["gathered"] == r1["gathered"]
+    (s0, seed0), (s1, seed1) = r0["gathered"]
+    assert s0 != s1 and (seed0, seed1) == (r0["plan"]["seed"], r1["plan"]["seed"])
+    assert r0["cfg"] == r1["cfg"] == (2, "dp2")           # global batch = B * world
+    assert r0["plan"]["global_batch"] == 2 and r0["plan"]["parallelism"] == "dp2"
 
 
 def test_single_rank_needs_no_process_group():
@@ -74,13 +92,22 @@ def test_single_rank_needs_no_process_group():
 
 def test_clock_sample_summary():
     c = bench.ClockSampler(0)
-    c.lines = ["0, 1965, 1965, 700.5, 0x0, Not Active, Not Active, Not Active, Not Active",
-               "0, 1800, 1965, 990.1, 0x4, Not Active, Not Active, Not Active, Active",
-               "0, 1900, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active",
-               "garbage"]
+    c.sm_max = 1965.0
+    c.samples = [(1965.0, 700.5, 0x0), (1800.0, 990.1, 0x4), (1900.0, 950.0, 0x4 | 0x1)]
     s = c.summary()
-    assert s["sm_mhz"] == 1900 and s["sm_max_mhz"] == 1965
-    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
+    assert s["sm_mhz"] == 1900 and s["sm_max_mhz"] == 1965 and s["sm_mhz_min"] == 1800
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3 and s["power_w_max"] == 990.1
+    c.samples = [(1500.0, 500.0, 0x8 | 0x40 | 0x20)]
+    assert c.summary()["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+
+
+def test_clock_sampler_reports_why_it_has_no_samples():
+    # No GPU here: NVML cannot start, and the summary says so instead of inventing clocks.
+    with bench.ClockSampler(0, period_s=0.001) as c:
+        pass
+    s = c.summary()
+    if s["samples"] == 0:
+        assert s["sm_mhz"] is None and "error" in s
 
 
 def test_peaks_and_recorded_traffic(tmp_path, monkeypatch):
