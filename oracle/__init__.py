@@ -14,14 +14,16 @@ the pages (see each function's docstring for the passage it follows):
   create_block_mask(...)                        per-tile partial / full lists
   attention(q, k, v, mask_mod, score_mod)       softmax(score_mod(scale*QK^T)
                                                 masked) @ V, and logsumexp
-  attention_backward(q, k, v, dO, ...)          dQ, dK, dV of that definition (for
-                                                the backward pass, not built yet)
+  attention_backward(q, k, v, dO, ...)          dQ, dK, dV of that definition
+  masked_softmax(scores, offset)                causal select + softmax over
+                                                materialised scores (the unfused chain)
 
 Every function is pinned by a "not gpu" test against facts the pages or the
 mathematics fix; where a function follows a reading of the pages (the composition
 order of soft-cap and ALiBi, for one), the pin checks that reading.
 """
 from .backward import attention_backward, make_score_mod_grad, soft_cap_grad  # noqa: F401
+from .masked_softmax import masked_softmax, causal_keep, finfo_min, BF16_MIN, FP16_MIN  # noqa: F401
 from .attention import (  # noqa: F401
     causal, sliding_window, document, conjunction, all_true, make_mask_mod,
     dense_mask, soft_cap, alibi, alibi_slopes, compose_score_mods,

@@ -13,6 +13,12 @@ Recipe (the same for every workload):
     (batch, heads, sequence, head_dim) is the one FlexAttention shares with
     scaled_dot_product_attention ("How to Use FlexAttention on Apple Silicon",
     Setup section).
+  * The masked-softmax workloads take materialised scores: i.i.d. N(0, 1) float32 (the
+    distribution of scale * q k^T for unit-variance q and k), drawn from
+    ``torch.Generator('cpu').manual_seed(seed)`` with shape (B, H, Q, K) and rounded to
+    bf16.  Q is a chunk of 1024 query rows that closes a context of K keys, so the causal
+    offset is K - Q (the 8K and 32K sequences of "Fuse the causal mask into the SDPA
+    fallback softmax", MLX pull request 3919).
   * The document-packed workload splits T = 8192 positions into 4 documents of
     seeded random lengths, each at least 512 long: three cut points drawn from
     ``numpy.random.default_rng(seed).integers(0, 6145, 3)`` and sorted give the
@@ -137,3 +143,40 @@ def three_doc_ids_from_page(S: int = 8192) -> np.ndarray:
     d[2048:] = 1
     d[5000:] = 2
     return d
+
+
+@dataclasses.dataclass(frozen=True)
+class SoftmaxWorkload:
+    """Causal-masked softmax over a (B, H, Q, K) tensor of materialised scores."""
+    name: str
+    B: int
+    H: int
+    Q: int
+    K: int
+    offset: int           # query row q sees keys kv <= q + offset
+    dtype: str = "bf16"
+    seed: int = 0
+
+    def scaled(self, Q: Optional[int] = None, K: Optional[int] = None,
+               H: Optional[int] = None) -> "SoftmaxWorkload":
+        Q = Q or self.Q
+        K = K or self.K
+        return dataclasses.replace(self, Q=Q, K=K, H=H or self.H, offset=K - Q)
+
+
+SOFTMAX_WORKLOADS = [
+    SoftmaxWorkload("masked_softmax_b1h8_q1024_k32768_bf16", B=1, H=8, Q=1024, K=32768,
+                    offset=32768 - 1024, seed=31),
+    SoftmaxWorkload("masked_softmax_b1h8_q1024_k8192_bf16", B=1, H=8, Q=1024, K=8192,
+                    offset=8192 - 1024, seed=32),
+]
+SOFTMAX_BY_NAME = {w.name: w for w in SOFTMAX_WORKLOADS}
+
+
+def make_scores(w: SoftmaxWorkload, seed: Optional[int] = None):
+    """Materialised scores on the CPU in the workload's dtype, as the module doc says."""
+    import torch
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    t = torch.randn((w.B, w.H, w.Q, w.K), generator=g, dtype=torch.float32)
+    return t.to(torch_dtype(w.dtype))
