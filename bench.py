@@ -379,6 +379,57 @@ def time_forward(w: wl.Workload, steps: int, warmup: int, world: int, rank: int,
             "lse": lse, "bm": bm}
 
 
+def softmax_bytes(w: wl.SoftmaxWorkload) -> int:
+    """Algorithmic bytes of one fused masked softmax: the live scores read once (scores past
+    the causal boundary are never needed) and every probability written once, 2 bytes each."""
+    q = np.arange(w.Q, dtype=np.int64)
+    live = np.clip(q + w.offset + 1, 0, w.K).sum()
+    return int(2 * w.B * w.H * (live + w.Q * w.K))
+
+
+def time_masked_softmax(w: wl.SoftmaxWorkload, steps: int, warmup: int, world: int, dev) -> dict:
+    """Time the fused causal-masked softmax (CUDA events on the launching stream, L2 flushed
+    before each step) and report its HBM roofline."""
+    import torch
+    import block_sparse_masked_x128_b200 as fa
+
+    scores = wl.make_scores(w).to(dev)
+    out = torch.empty_like(scores)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.zero_()
+        fa.masked_softmax(scores, w.offset, out=out)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    with ClockSampler(dev.index) as clocks:
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            fa.masked_softmax(scores, w.offset, out=out)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if fa.fa_masked_softmax_status() != fa.FA_OK:
+        raise RuntimeError("a masked-softmax wait timed out")
+    per = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    t_max = max_over_ranks(sum(per), world, dev)
+    nbytes = softmax_bytes(w)
+    peaks = read_peaks()
+    achieved = nbytes / (statistics.mean(per) * 1e-3) / 1e9
+    return {"metric": "fused causal-masked softmax GB/s (live scores read + probabilities written)",
+            "value": world * nbytes * steps / (t_max * 1e-3) / 1e9, "unit": "GB/s",
+            "ms_per_step": t_max / steps, "bytes_per_step": nbytes, "gpu_launches": steps,
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "Q": w.Q, "K": w.K,
+                       "offset": w.offset, "dtype": w.dtype},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": None, "peak_source": peaks["source"] + " hbm_gbs",
+                         "kernel": "masked_softmax_kernel"},
+            "clocks": clocks.summary()}
+
+
 def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
     import torch
     import block_sparse_masked_x128_b200 as fa
@@ -495,6 +546,13 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
             del o
             torch.cuda.empty_cache()
         res["per_workload"] = per
+
+    # The rows after the forward: each timed on its own headline workload.
+    if not args.no_per_workload:
+        res["next_rows"] = {
+            "masked_softmax": time_masked_softmax(wl.SOFTMAX_WORKLOADS[0], args.steps, args.warmup,
+                                                  world, dev)}
+        torch.cuda.empty_cache()
 
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         q, k, v = wl.make_qkv(w, seed=rank_plan(w, world, rank)["seed"])

@@ -41,12 +41,13 @@ FA_DTYPE_BF16 = 1
 
 EXPORTED = ("fa_create_block_mask", "fa_forward", "fa_block_mask_get", "fa_get_device_status",
             "fa_destroy_block_mask", "fa_status_string", "fa_last_error_message",
-            "fa_create_block_mask_noalloc", "fa_debug_set_stall")
+            "fa_create_block_mask_noalloc", "fa_debug_set_stall", "fa_masked_softmax",
+            "fa_masked_softmax_status")
 
 
 class FaMaskParams(ctypes.Structure):
     _fields_ = [("window", ctypes.c_int32), ("doc_id", ctypes.c_void_p),
-                ("separate_full_blocks", ctypes.c_int32)]
+                ("separate_full_blocks", ctypes.c_int32), ("dq_kv_order", ctypes.c_int32)]
 
 
 class FaScoreParams(ctypes.Structure):
@@ -95,6 +96,11 @@ _lib.fa_last_error_message.argtypes = []
 _lib.fa_last_error_message.restype = ctypes.c_char_p
 _lib.fa_debug_set_stall.argtypes = [ctypes.c_int32]
 _lib.fa_debug_set_stall.restype = _status
+_lib.fa_masked_softmax.argtypes = [ctypes.POINTER(FaTensor), ctypes.c_uint32, ctypes.c_int64,
+                                   ctypes.POINTER(FaTensor), ctypes.c_void_p]
+_lib.fa_masked_softmax.restype = _status
+_lib.fa_masked_softmax_status.argtypes = [ctypes.c_void_p]
+_lib.fa_masked_softmax_status.restype = _status
 
 
 class FaError(RuntimeError):
@@ -194,6 +200,17 @@ def fa_destroy_block_mask(block_mask: int) -> None:
     _lib.fa_destroy_block_mask(block_mask)
 
 
+def fa_masked_softmax(scores: FaTensor, mask_kind: int, offset: int, probs: FaTensor,
+                      stream=None) -> None:
+    _check(_lib.fa_masked_softmax(ctypes.byref(scores), mask_kind, offset, ctypes.byref(probs),
+                                  _stream_ptr(stream)), "fa_masked_softmax")
+
+
+def fa_masked_softmax_status(stream=None) -> int:
+    """Synchronise the stream and return FA_OK or FA_ERR_TIMEOUT for the softmax kernels."""
+    return _lib.fa_masked_softmax_status(_stream_ptr(stream))
+
+
 def fa_debug_set_stall(enable: bool) -> None:
     """Test hook: make every later forward's bounded K wait run out (see the C header)."""
     _check(_lib.fa_debug_set_stall(1 if enable else 0), "fa_debug_set_stall")
@@ -273,7 +290,8 @@ def check_doc_id(doc_id, KV_LEN: int, device) -> None:
 
 def create_block_mask(mask_kind: int, B: Optional[int], H: Optional[int], Q_LEN: int, KV_LEN: int,
                       *, window: int = 0, doc_id=None, separate_full_blocks: bool = True,
-                      BLOCK_SIZE: int = 128, device=None, stream=None) -> BlockMask:
+                      dq_kv_order: bool = True, BLOCK_SIZE: int = 128, device=None,
+                      stream=None) -> BlockMask:
     """Build a block mask on the current CUDA device (B or H of None broadcasts)."""
     import torch
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
@@ -282,7 +300,8 @@ def create_block_mask(mask_kind: int, B: Optional[int], H: Optional[int], Q_LEN:
         # The C ABI reads KV_LEN ids through a bare pointer: check what it cannot.
         check_doc_id(doc_id, KV_LEN, dev)
         doc_ptr = doc_id.data_ptr()
-    params = FaMaskParams(int(window), doc_ptr, 1 if separate_full_blocks else 0)
+    params = FaMaskParams(int(window), doc_ptr, 1 if separate_full_blocks else 0,
+                          1 if dq_kv_order else 0)
     with torch.cuda.device(dev):
         h = fa_create_block_mask(int(mask_kind), params, int(B or 0), int(H or 0), int(Q_LEN),
                                  int(KV_LEN), int(BLOCK_SIZE), stream)
@@ -321,3 +340,19 @@ def flex_attention(q, k, v, block_mask: BlockMask, *, score_mod: int = FA_SCORE_
                    lse.data_ptr() if lse is not None else None, stream)
     return out, lse
 
+
+
+def masked_softmax(scores, offset: Optional[int] = None, *, causal: bool = True, out=None,
+                   stream=None):
+    """softmax(where(q + offset >= kv, scores, finfo.min)) over the last axis of a
+    (B, H, Q, K) fp16/bf16 CUDA tensor, in one fused kernel; offset defaults to K - Q.
+    ``causal=False`` gives the plain softmax.  ``out`` may be ``scores`` (in place)."""
+    import torch
+    if offset is None:
+        offset = scores.shape[3] - scores.shape[2]
+    if out is None:
+        out = torch.empty_like(scores)
+    with torch.cuda.device(scores.device):
+        fa_masked_softmax(fa_tensor(scores), FA_MASK_CAUSAL if causal else 0, int(offset),
+                          fa_tensor(out), stream)
+    return out

@@ -27,7 +27,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libfa_b200.so")
 TRACE_LIB = os.path.join(LIBDIR, "libfa_b200_trace.so")
-SOURCES = ["api.cu", "mask_builder.cu", "attn_fwd.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "mask_builder.cu", "attn_fwd.cu", "noalloc.cu", "masked_softmax.cu", "attn_bwd.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

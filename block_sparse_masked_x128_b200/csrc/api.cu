@@ -226,10 +226,20 @@ fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* par
     const size_t o_kvn = take(BH * QB * 4), o_kvi = take(BH * QB * KVB * 4);
     const size_t o_fn = take(BH * QB * 4), o_fi = take(BH * QB * KVB * 4);
     const bool has_doc = (mask_kind & FA_MASK_DOCUMENT) != 0;
-    const size_t o_doc = take(has_doc ? (size_t)KV_LEN * 4 : 0);
+    // The copy of doc_id is padded to whole blocks (the forward reads ids by 128-key tile).
+    const size_t doc_pad = (size_t)KVB * fa::kBlock;
+    const size_t o_doc = take(has_doc ? doc_pad * 4 : 0);
     const size_t o_dst = take(has_doc ? (size_t)(QB > KVB ? QB : KVB) * 3 * 4 : 0);
     const size_t o_sc = take(BH * NP * 8), o_scost = take(BH * NP * 4);
     const size_t o_se = take(BH * NP * KVB * 4), o_so = take(BH * NP * 4);
+    // Backward metadata: transposed lists, the dK/dV kernel's kv-major units, the dQ units.
+    const size_t n_kv = BH * KVB, n_q = BH * QB, n_tiles = BH * QB * KVB;
+    const size_t o_qn = take(n_kv * 4), o_qi = take(n_tiles * 4), o_fqn = take(n_kv * 4),
+                 o_fqi = take(n_tiles * 4);
+    const size_t o_kvc = take(n_kv * 4), o_kvcost = take(n_kv * 4), o_kve = take(n_tiles * 4),
+                 o_kvo = take(n_kv * 4);
+    const size_t o_dqc = take(n_q * 4), o_dqcost = take(n_q * 4), o_dqe = take(n_tiles * 4),
+                 o_dqo = take(n_q * 4);
     // Status word, then the forward's unit counters (two words per slot), all zero.
     const size_t ctr_bytes = 4 + (size_t)fa::kSchedCtrSlots * 8;
     const size_t o_status = take(ctr_bytes);
@@ -263,6 +273,10 @@ fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* par
     m->sched_cost = reinterpret_cast<int32_t*>(b8 + o_scost);
     m->sched_entries = reinterpret_cast<int32_t*>(b8 + o_se);
     m->sched_order = reinterpret_cast<int32_t*>(b8 + o_so);
+    auto at = [&](size_t o) { return reinterpret_cast<int32_t*>(b8 + o); };
+    m->dq_kv_order = params ? (params->dq_kv_order ? 1 : 0) : 1;
+    m->bwd = fa::BwdMeta{at(o_qn),  at(o_qi),     at(o_fqn), at(o_fqi), at(o_kvc),    at(o_kvcost),
+                         at(o_kve), at(o_kvo),    at(o_dqc), at(o_dqcost), at(o_dqe), at(o_dqo)};
     m->status = reinterpret_cast<int32_t*>(b8 + o_status);
     m->sched_ctr = m->status + 1;
 
@@ -277,6 +291,9 @@ fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* par
         (e = cudaMemcpyAsync(m->doc, params->doc_id, (size_t)KV_LEN * 4, cudaMemcpyDefault, st)) !=
             cudaSuccess)
         return bail(e, "copy of doc_id");
+    if (has_doc && doc_pad > (size_t)KV_LEN &&
+        (e = cudaMemsetAsync(m->doc + KV_LEN, 0, (doc_pad - KV_LEN) * 4, st)) != cudaSuccess)
+        return bail(e, "padding of doc_id");
     fa::MaskSpec spec;
     spec.kind = mask_kind;
     spec.window = window;
@@ -290,6 +307,9 @@ fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* par
                               m->full_idx, m->doc_stats, m->sched_count, m->sched_cost,
                               m->sched_entries, m->sched_order, st);
     if (e != cudaSuccess) return bail(e, "mask-builder launch");
+    e = fa::launch_backward_metadata(QB, KVB, (int)BH, m->dq_kv_order, m->kv_num, m->kv_idx,
+                                     m->full_num, m->full_idx, m->bwd, st);
+    if (e != cudaSuccess) return bail(e, "backward-metadata launch");
     *out_mask = m;
     return ok();
 }
@@ -361,8 +381,6 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
     if (out->S != q->S) return fail(FA_ERR_INVALID_ARG, "out must have q's S");
     if (q->D != 64 && q->D != 128)
         return fail(FA_ERR_UNSUPPORTED, "head_dim %lld: only 64 and 128 are implemented", (long long)q->D);
-    if ((q->S % fa::kBlock) != 0 || (k->S % fa::kBlock) != 0)
-        return fail(FA_ERR_UNSUPPORTED, "Q_LEN and KV_LEN must be multiples of 128");
     const uint32_t known = FA_SCORE_SOFTCAP | FA_SCORE_ALIBI;
     if (score_mod_kind & ~known) return fail(FA_ERR_INVALID_ARG, "unknown score_mod_kind bits 0x%x", score_mod_kind);
     if ((score_mod_kind & FA_SCORE_SOFTCAP) && (!params || !(params->softcap > 0.f)))
@@ -443,6 +461,55 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
         return fa::launch_attn_fwd(p, (int)q->D, q->dtype == FA_DTYPE_BF16, (int)score_mod_kind,
                                    tq, tk, tv, grid, st);
     });
+}
+
+fa_status_t fa_masked_softmax(const fa_tensor_t* scores, uint32_t mask_kind, int64_t offset,
+                              fa_tensor_t* probs, void* stream) {
+    fa_status_t s;
+    if ((s = check_tensor(scores, "scores")) != FA_OK) return s;
+    if ((s = check_tensor(probs, "probs")) != FA_OK) return s;
+    if (probs->dtype != scores->dtype) return fail(FA_ERR_INVALID_ARG, "scores and probs must share one dtype");
+    if (probs->B != scores->B || probs->H != scores->H || probs->S != scores->S || probs->D != scores->D)
+        return fail(FA_ERR_INVALID_ARG, "scores and probs must have the same shape");
+    if (mask_kind != 0 && mask_kind != FA_MASK_CAUSAL)
+        return fail(FA_ERR_UNSUPPORTED, "mask_kind 0x%x: the fused softmax takes FA_MASK_CAUSAL or 0", mask_kind);
+    const int64_t K = scores->D;
+    if ((K % 8) != 0) return fail(FA_ERR_UNSUPPORTED, "K=%lld: rows must be whole 16-byte vectors (K %% 8 == 0)", (long long)K);
+    if (K > fa::masked_softmax_max_keys())
+        return fail(FA_ERR_UNSUPPORTED, "K=%lld above the %d keys a row may hold", (long long)K, fa::masked_softmax_max_keys());
+    if (scores->B > 0x7fffffff || scores->H > 0x7fffffff || scores->S > 0x7fffffff)
+        return fail(FA_ERR_UNSUPPORTED, "extent above 2^31 - 1");
+    if (probs->data != scores->data) {
+        // Distinct buffers must not overlap (the same buffer with the same strides is fine:
+        // every row is read before it is written).
+    } else {
+        for (int i = 0; i < 3; ++i)
+            if (probs->stride[i] != scores->stride[i])
+                return fail(FA_ERR_INVALID_ARG, "in-place softmax needs probs and scores to share strides");
+    }
+    if (scores->B == 0 || scores->H == 0 || scores->S == 0) return ok();
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if ((s = fa::check_device_memory(scores->data, dev, "scores")) != FA_OK) return s;
+    if ((s = fa::check_device_memory(probs->data, dev, "probs")) != FA_OK) return s;
+    const int nsm = sm_count(dev);
+    if (nsm <= 0) return fail(FA_ERR_CUDA, "could not read the SM count");
+    e = fa::launch_masked_softmax_checked(scores->data, probs->data, scores->stride, probs->stride,
+                                          (int)scores->B, (int)scores->H, (int)scores->S, (int)K,
+                                          offset, mask_kind == FA_MASK_CAUSAL,
+                                          scores->dtype == FA_DTYPE_BF16, nsm,
+                                          static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "masked-softmax launch");
+    return ok();
+}
+
+fa_status_t fa_masked_softmax_status(void* stream) {
+    int32_t h = 0;
+    cudaError_t e = fa::masked_softmax_status(static_cast<cudaStream_t>(stream), &h);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the masked-softmax status word");
+    if (h != 0) return fail(FA_ERR_TIMEOUT, "a masked-softmax wait ran past its limit (status %d)", h);
+    return ok();
 }
 
 // Test hook for failure detection (see the header): read by every later fa_forward.

@@ -60,6 +60,68 @@ struct FwdParams {
     int32_t stall_loads;          // test hook: the TMA warp stops after the first Q tiles
 };
 
+// Backward metadata of a mask (all int32, maskBH = stored B * H):
+//   q_num, fq_num [maskBH][KVB]; q_idx, fq_idx [maskBH][KVB][QB]: per kv block, the query
+//     blocks whose tile is partial / full, ascending, zero padded (the transposed lists);
+//   kv_count, kv_cost, kv_order [maskBH][KVB]; kv_entries [maskBH][KVB][QB]: the dK/dV
+//     kernel's units, one per kv block: entries query block | kLive0 (| kFull0) ascending,
+//     units ranked by cost (longest first);
+//   dq_count, dq_cost, dq_order [maskBH][QB]; dq_entries [maskBH][QB][KVB]: the dQ kernel's
+//     units, one per query block: kv block | kLive0 (| kFull0) in the mask's dQ write order.
+struct BwdMeta {
+    int32_t *q_num, *q_idx, *fq_num, *fq_idx;
+    int32_t *kv_count, *kv_cost, *kv_entries, *kv_order;
+    int32_t *dq_count, *dq_cost, *dq_entries, *dq_order;
+};
+
+cudaError_t launch_backward_metadata(int QB, int KVB, int maskBH, int dq_descending,
+                                     const int32_t* kv_num, const int32_t* kv_idx,
+                                     const int32_t* full_num, const int32_t* full_idx,
+                                     const BwdMeta& m, cudaStream_t stream);
+
+// Kernel parameters of the backward kernels (attn_bwd.cu).  A unit is one kv block (dK/dV
+// kernel) or one query block (dQ kernel) of one (b, h); its entries are the tiles it visits.
+struct BwdParams {
+    int32_t B, H, Q_LEN, KV_LEN, QB, KVB;
+    int32_t maskB, maskH;
+    int32_t units_per_bh;         // KVB (dK/dV kernel) or QB (dQ kernel)
+    int32_t entries_stride;       // QB (dK/dV kernel) or KVB (dQ kernel)
+    int32_t n_units;              // units_per_bh * B * H
+    int32_t head_major;           // 1: units of one (b, h) are handed out together
+    uint32_t mask_kind;
+    int32_t window;
+    uint32_t score_kind;
+    const int32_t* doc_id;
+    const int32_t* order;         // [maskB*maskH][units_per_bh]  units by descending cost
+    const int32_t* count;         // [maskB*maskH][units_per_bh]  entries per unit
+    const int32_t* entries;       // [maskB*maskH][units_per_bh][entries_stride]
+    float scale;
+    float scale_log2;             // scale * log2(e)
+    float softcap_log2;           // softcap * log2(e)
+    float inv_softcap_scale;      // scale / softcap
+    const float* alibi_slopes;    // device [H] or null (then 2^(-8(h+1)/H))
+    const float* lse_log2;        // workspace [B*H][q_pad]: lse * log2(e), +inf without keys
+    const float* delta;           // workspace [B*H][q_pad]: rowsum(dO * O)
+    int32_t q_pad;                // QB * 128
+    void* grad0;                  // dK/dV kernel: dK; dQ kernel: dQ
+    void* grad1;                  // dK/dV kernel: dV; dQ kernel: unused
+    int64_t grad0_stride[3];      // B, H, S strides in elements
+    int64_t grad1_stride[3];
+    int32_t* status;
+    int32_t* sched_ctr;
+};
+
+cudaError_t launch_bwd_preprocess(const void* out, const int64_t out_stride[3], const void* dout,
+                                  const int64_t dout_stride[3], const float* lse, int B, int H,
+                                  int Q_LEN, int q_pad, int D, bool bf16, float* lse_log2,
+                                  float* delta, cudaStream_t stream);
+cudaError_t launch_attn_bwd_dkdv(const BwdParams& p, int D, bool bf16, int score_kind,
+                                 const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                 const CUtensorMap& tdo, int grid, cudaStream_t stream);
+cudaError_t launch_attn_bwd_dq(const BwdParams& p, int D, bool bf16, int score_kind,
+                               const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const CUtensorMap& tdo, int grid, cudaStream_t stream);
+
 cudaError_t launch_mask_build(const MaskSpec& spec, int separate_full, int maskBH, int NP,
                               int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
                               int32_t* full_idx, int32_t* doc_stats, int32_t* sched_count,
@@ -79,6 +141,15 @@ fa_status_t record_ok();
 cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, int score_kind,
                             const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             int grid, cudaStream_t stream);
+
+// Causal-masked softmax over materialised scores (masked_softmax.cu).
+struct SoftmaxParams;
+int masked_softmax_max_keys();
+cudaError_t launch_masked_softmax_checked(const void* in, void* out, const int64_t in_stride[3],
+                                          const int64_t out_stride[3], int B, int H, int Q, int K,
+                                          int64_t offset, bool causal, bool bf16, int num_sms,
+                                          cudaStream_t stream);
+cudaError_t masked_softmax_status(cudaStream_t stream, int32_t* out);
 
 // Counter pairs per mask for the forward's run-time unit hand-out: each launch takes the
 // next pair, so up to this many forwards may run at once on one mask.
@@ -105,6 +176,8 @@ struct fa_block_mask {
     int32_t* sched_entries;
     int32_t* sched_order;
     int32_t* status;
+    int32_t dq_kv_order;      // 1: dQ accumulates kv blocks in descending order, 0: ascending
+    fa::BwdMeta bwd;
     int32_t* sched_ctr;       // fa::kSchedCtrSlots pairs of unit counters after the status word
     // Round-robin pick of a counter pair per forward.  ctr_event[s] is recorded after the
     // last forward that used pair s; the next forward on pair s waits for it on the GPU, so

@@ -1,0 +1,338 @@
+// masked_softmax.cu -- the causal-masked softmax over materialised scores, fused.
+//
+// What it computes ("Fuse the causal mask into the SDPA fallback softmax", MLX pull request
+// 3919, Summary and Description): the chain
+//     keep = q + offset >= kv;  x = keep ? score : finfo(dtype).min;  probs = softmax(x)
+// in one pass over memory.  The select is applied where the scores are read, so the
+// per-element arithmetic is the plain softmax's on the selected values: the result is
+// bit-identical to running this kernel without the mask on where(keep, scores, finfo.min),
+// and masked entries are exactly zero (exp(finfo.min - max) underflows).  Scores behind the
+// causal boundary are never read: their selected value does not depend on them.
+//
+// Organisation (HBM-bound; one persistent CTA of 512 threads per SM):
+//   * rows (b, h, q) are dealt round robin to the CTAs;
+//   * thread 0 stages each row's live prefix into shared memory with one cp.async.bulk load,
+//     a ring of `stages` row buffers deep (so up to stages - 1 rows are in flight while one
+//     is computed), completing on one mbarrier per buffer;
+//   * all threads then hold the row in registers (thread t owns the 16-byte vectors
+//     t, t + 512, ...), take the row max and the row sum of e = 2^((x - max) log2 e) with
+//     warp shuffles and a fixed-order cross-warp step, and write p = e / sum back over the
+//     buffer as 16-bit values;
+//   * thread 0 writes the row out with one cp.async.bulk store; the buffer is reloaded once
+//     that store has read it (bulk wait_group.read, one row behind).
+// Every reduction has the same order in the masked and the unmasked run, which is what
+// makes them bit-identical.  Waits are bounded: a wait that runs out sets the status word,
+// and the CTA drains its own copies before it returns.
+#include <cfloat>
+
+#include <cuda_fp16.h>
+
+#include "fa_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+struct SoftmaxParams {
+    const uint16_t* in;
+    uint16_t* out;
+    int64_t in_stride[3];   // b, h, q strides in elements (the key stride is 1)
+    int64_t out_stride[3];
+    int32_t B, H, Q, K;
+    int64_t offset;         // query row q keeps keys kv <= q + offset
+    int32_t causal;
+    int64_t rows;           // B * H * Q
+    int32_t stages;
+    uint32_t stage_bytes;   // K * 2 rounded up to 128
+    int32_t* status;
+};
+
+namespace {
+
+constexpr int kSmThreads = 512;
+constexpr int kSmWarps = kSmThreads / 32;
+constexpr uint64_t kSmWaitLimitNs = 2000000000ull;
+constexpr float kSmLog2e = 1.4426950408889634f;
+
+__device__ int32_t g_softmax_status;
+
+template <bool BF16>
+__device__ __forceinline__ float dtype_min() {
+    // finfo(bfloat16).min = -(2 - 2^-7) * 2^127 and finfo(float16).min = -65504, as float.
+    return BF16 ? -3.38953138925153547590e38f : -65504.0f;
+}
+
+template <bool BF16>
+__device__ __forceinline__ float to_f32(uint32_t bits16) {
+    return BF16 ? __uint_as_float(bits16 << 16) : __half2float(__ushort_as_half((unsigned short)bits16));
+}
+
+__device__ __forceinline__ int64_t live_keys(const SoftmaxParams& p, int64_t q) {
+    if (!p.causal) return p.K;
+    int64_t n = q + p.offset + 1;
+    return n < 0 ? 0 : (n > p.K ? p.K : n);
+}
+
+__device__ __forceinline__ void row_coords(const SoftmaxParams& p, int64_t r, int64_t& b, int64_t& h,
+                                           int64_t& q) {
+    q = r % p.Q;
+    const int64_t bh = r / p.Q;
+    h = bh % p.H;
+    b = bh / p.H;
+}
+
+// Bytes the bulk load brings for row r: its live prefix rounded up to 16 bytes (K is a
+// multiple of 8, so the rounding stays inside the row).
+__device__ __forceinline__ uint32_t load_bytes(const SoftmaxParams& p, int64_t r) {
+    int64_t b, h, q;
+    row_coords(p, r, b, h, q);
+    const int64_t n = live_keys(p, q);
+    return (uint32_t)(((n + 7) & ~7ll) * 2);
+}
+
+__device__ __forceinline__ void issue_row_load(const SoftmaxParams& p, int64_t r, uint32_t dst,
+                                               uint32_t bar) {
+    int64_t b, h, q;
+    row_coords(p, r, b, h, q);
+    const uint32_t bytes = load_bytes(p, r);
+    mbar_arrive_expect_tx(bar, bytes);
+    if (bytes > 0)
+        bulk_load(dst, p.in + b * p.in_stride[0] + h * p.in_stride[1] + q * p.in_stride[2], bytes, bar);
+}
+
+// Bounded wait by every thread; the outcome is made block-uniform.
+__device__ __forceinline__ bool block_wait(uint32_t bar, uint32_t parity) {
+    bool ok = mbar_try_wait(bar, parity);
+    if (!ok) {
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t it = 1;; ++it) {
+            if (mbar_try_wait(bar, parity)) { ok = true; break; }
+            if ((it & 127u) == 0u && global_timer_ns() - t0 > kSmWaitLimitNs) break;
+        }
+    }
+    return __syncthreads_and(ok ? 1 : 0) != 0;
+}
+
+template <bool BF16, int VPT>
+__global__ void __launch_bounds__(kSmThreads, 1) masked_softmax_kernel(const __grid_constant__ SoftmaxParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                               ~static_cast<uintptr_t>(127));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bars = sbase + (uint32_t)p.stages * p.stage_bytes;
+    float* red = reinterpret_cast<float*>(smem + (size_t)p.stages * p.stage_bytes + 8 * p.stages);
+    float* red_max = red;
+    float* red_sum = red + kSmWarps;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t grid = gridDim.x;
+
+    if (tid == 0) {
+        for (int s = 0; s < p.stages; ++s) mbar_init(bars + 8u * s, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // Rows of this CTA: blockIdx.x + k * grid, k = 0, 1, ...; row k lives in buffer k % stages.
+    const int64_t my_rows = (p.rows > blockIdx.x) ? (p.rows - blockIdx.x + grid - 1) / grid : 0;
+    int64_t issued = 0;   // rows whose load thread 0 has issued
+    if (tid == 0) {
+        for (; issued < my_rows && issued < p.stages; ++issued)
+            issue_row_load(p, blockIdx.x + issued * grid, sbase + (uint32_t)issued * p.stage_bytes,
+                           bars + 8u * (uint32_t)issued);
+    }
+    const float kMasked = dtype_min<BF16>();
+    int64_t k = 0;
+    bool ok = true;
+    for (; k < my_rows; ++k) {
+        const int s = (int)(k % p.stages);
+        const uint32_t buf = sbase + (uint32_t)s * p.stage_bytes;
+        if (!block_wait(bars + 8u * s, (uint32_t)((k / p.stages) & 1))) { ok = false; break; }
+        const int64_t r = blockIdx.x + k * grid;
+        int64_t b, h, q;
+        row_coords(p, r, b, h, q);
+        const int64_t n_live = live_keys(p, q);
+        const uint16_t* srow = reinterpret_cast<const uint16_t*>(smem + (size_t)s * p.stage_bytes);
+
+        // Pass 1: the selected values in registers, and the row max.
+        float x[VPT * 8];
+        float m = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+            const int64_t e0 = 8ll * (tid + kSmThreads * j);
+            if (e0 >= p.K) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[8 * j + i] = -INFINITY;   // past the row: no key
+            } else if (e0 >= n_live) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[8 * j + i] = kMasked;
+                m = fmaxf(m, kMasked);
+            } else {
+                const uint4 raw = *reinterpret_cast<const uint4*>(srow + e0);
+                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float v = to_f32<BF16>((w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+                    x[8 * j + i] = (e0 + i < n_live) ? v : kMasked;
+                    m = fmaxf(m, x[8 * j + i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+        if (lane == 0) red_max[warp] = m;
+        __syncthreads();
+        m = red_max[0];
+#pragma unroll
+        for (int w = 1; w < kSmWarps; ++w) m = fmaxf(m, red_max[w]);
+
+        // Pass 2: e = 2^((x - m) log2 e) and the row sum, in a fixed order.  A vector wholly
+        // past the causal boundary holds exp(finfo.min - m) = 0 unless the whole row is
+        // masked (m == finfo.min), where it is computed like any other.
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+            const int64_t e0 = 8ll * (tid + kSmThreads * j);
+            if (e0 >= p.K) continue;
+            if (e0 >= n_live && m != kMasked) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[8 * j + i] = 0.f;
+                continue;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float e = ex2_approx((x[8 * j + i] - m) * kSmLog2e);
+                x[8 * j + i] = e;
+                sum += e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o);
+        if (lane == 0) red_sum[warp] = sum;
+        __syncthreads();
+        sum = red_sum[0];
+#pragma unroll
+        for (int w = 1; w < kSmWarps; ++w) sum += red_sum[w];
+        const float inv = 1.0f / sum;
+
+        // Pass 3: p = e / sum as 16-bit values over the buffer, then one bulk store.
+        uint16_t* wrow = reinterpret_cast<uint16_t*>(smem + (size_t)s * p.stage_bytes);
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+            const int64_t e0 = 8ll * (tid + kSmThreads * j);
+            if (e0 >= p.K) continue;
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[i] = pack2<BF16>(x[8 * j + 2 * i] * inv, x[8 * j + 2 * i + 1] * inv);
+            *reinterpret_cast<uint4*>(wrow + e0) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_store(p.out + b * p.out_stride[0] + h * p.out_stride[1] + q * p.out_stride[2], buf,
+                       (uint32_t)(p.K * 2));
+            bulk_commit();
+            // Refill the buffer of the previous row once its store has read it.
+            if (k >= 1 && issued < my_rows) {
+                bulk_wait_read<1>();
+                fence_proxy_async_smem();
+                const int ps = (int)((k - 1) % p.stages);
+                issue_row_load(p, blockIdx.x + issued * grid, sbase + (uint32_t)ps * p.stage_bytes,
+                               bars + 8u * (uint32_t)ps);
+                ++issued;
+            }
+        }
+    }
+    if (tid == 0) {
+        if (!ok) {
+            atomicExch(p.status, 1);
+            // Let the loads already issued land before the CTA's shared memory goes away.
+            for (int64_t kk = k; kk < issued; ++kk) {
+                const uint32_t bar = bars + 8u * (uint32_t)(kk % p.stages);
+                const uint32_t par = (uint32_t)((kk / p.stages) & 1);
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(bar, par) && global_timer_ns() - t0 < kSmWaitLimitNs) {
+                }
+            }
+        }
+        bulk_wait_all();
+    }
+}
+
+template <bool BF16, int VPT>
+cudaError_t launch_t(const SoftmaxParams& p, int grid, size_t smem, cudaStream_t stream) {
+    auto kern = masked_softmax_kernel<BF16, VPT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kSmThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int masked_softmax_max_keys() { return kSmThreads * 8 * 8; }
+
+cudaError_t launch_masked_softmax(SoftmaxParams p, bool bf16, int num_sms, cudaStream_t stream) {
+    // Row buffers: as many as fit in 200 KiB, 2 to 8.
+    p.stage_bytes = (uint32_t)(((int64_t)p.K * 2 + 127) & ~127ll);
+    int stages = (int)((200 * 1024) / p.stage_bytes);
+    stages = stages > 8 ? 8 : stages;
+    if (stages < 2) return cudaErrorInvalidValue;
+    p.stages = stages;
+    if (!p.status) {
+        void* addr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&addr, g_softmax_status);
+        if (e != cudaSuccess) return e;
+        p.status = static_cast<int32_t*>(addr);
+    }
+    const size_t smem = 128 + (size_t)stages * p.stage_bytes + 8 * stages + 2 * kSmWarps * sizeof(float);
+    const int grid = (int)(p.rows < num_sms ? p.rows : num_sms);
+    const int vpt_needed = (p.K + 8 * kSmThreads - 1) / (8 * kSmThreads);
+#define FA_SM_CASE(V)                                                              \
+    if (vpt_needed <= V)                                                           \
+        return bf16 ? launch_t<true, V>(p, grid, smem, stream)                     \
+                    : launch_t<false, V>(p, grid, smem, stream);
+    FA_SM_CASE(1)
+    FA_SM_CASE(2)
+    FA_SM_CASE(4)
+    FA_SM_CASE(8)
+#undef FA_SM_CASE
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_masked_softmax_checked(const void* in, void* out, const int64_t in_stride[3],
+                                          const int64_t out_stride[3], int B, int H, int Q, int K,
+                                          int64_t offset, bool causal, bool bf16, int num_sms,
+                                          cudaStream_t stream) {
+    SoftmaxParams p;
+    p.in = static_cast<const uint16_t*>(in);
+    p.out = static_cast<uint16_t*>(out);
+    for (int i = 0; i < 3; ++i) {
+        p.in_stride[i] = in_stride[i];
+        p.out_stride[i] = out_stride[i];
+    }
+    p.B = B;
+    p.H = H;
+    p.Q = Q;
+    p.K = K;
+    p.offset = offset;
+    p.causal = causal ? 1 : 0;
+    p.rows = (int64_t)B * H * Q;
+    p.stages = 0;
+    p.stage_bytes = 0;
+    p.status = nullptr;
+    return launch_masked_softmax(p, bf16, num_sms, stream);
+}
+
+// Read and clear the status word of the masked-softmax kernels (1 = a bounded wait ran out).
+cudaError_t masked_softmax_status(cudaStream_t stream, int32_t* out) {
+    void* addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_softmax_status);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyAsync(out, addr, 4, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && *out != 0) {
+        e = cudaMemsetAsync(addr, 0, 4, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    }
+    return e;
+}
+
+}  // namespace fa

@@ -77,6 +77,10 @@ typedef struct fa_mask_params {
     int32_t        separate_full_blocks;  /* 1: fully unmasked tiles go to the full_* lists so the
                                              kernel skips mask_mod there; 0: every live tile is
                                              listed as partial ("create_block_mask", Parameters)   */
+    int32_t        dq_kv_order;           /* order in which the backward accumulates each query
+                                             block's dQ over its kv blocks: 1 descending, 0
+                                             ascending ("create_block_mask", Parameters,
+                                             dq_kv_order; either order is deterministic)          */
 } fa_mask_params_t;
 
 typedef struct fa_score_params {
@@ -151,8 +155,9 @@ fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* par
  *   out         (B, H, Q_LEN, D), q's dtype, caller-owned
  *   lse         device fp32 [B][H][Q_LEN] contiguous, or NULL to skip it
  *
- * Supported now: D in {64, 128}; Q_LEN and KV_LEN multiples of 128 (else
- * FA_ERR_UNSUPPORTED).  q, k, v, out, lse and alibi_slopes must be memory of the current
+ * Supported: D in {64, 128} (else FA_ERR_UNSUPPORTED); any Q_LEN and KV_LEN >= 1 (a
+ * ragged last tile is loaded zero-filled, its keys past KV_LEN are masked and its rows past
+ * Q_LEN are not stored).  q, k, v, out, lse and alibi_slopes must be memory of the current
  * device (cudaMalloc or managed; host memory, pinned or not, gives FA_ERR_INVALID_ARG).  A query row with no allowed key gets out = 0, lse = -inf.
  * Device-side waits are bounded; a wait that runs out sets the mask's status word
  * (read it with fa_get_device_status) and the kernel returns early.
@@ -196,6 +201,39 @@ fa_status_t fa_create_block_mask_noalloc(uint32_t mask_kind, const fa_mask_param
                                          int32_t BLOCK_SIZE, int32_t* kv_num_blocks,
                                          int32_t* kv_indices, int32_t* full_kv_num_blocks,
                                          int32_t* full_kv_indices, void* stream);
+
+/*
+ * fa_masked_softmax -- the causal-masked softmax over materialised scores, in one kernel.
+ *
+ * probs[b,h,q,kv] = softmax over kv of  (q + offset >= kv ? scores[b,h,q,kv] : finfo.min)
+ *
+ * ("Fuse the causal mask into the SDPA fallback softmax", MLX pull request 3919, Summary and
+ * Description: the chain greater_equal -> where(finfo.min) -> softmax with the select folded
+ * into the softmax's loads.)  finfo.min is the scores dtype's lowest finite value; masked
+ * entries come out exactly 0, and a row whose keys are all masked is uniform, 1/K, as the
+ * chain gives.  The arithmetic is float32 (max, then the sum of 2^((x - max) log2 e), then
+ * e / sum rounded to the output dtype), with the same reduction order whether or not the
+ * mask is applied: with FA_MASK_CAUSAL the result is bit-identical to mask_kind 0 applied to
+ * where(keep, scores, finfo.min).  Scores past the causal boundary are never read.
+ *
+ *   scores     (B, H, Q, K) fp16 or bf16 in an fa_tensor_t (S = Q rows, D = K keys); the key
+ *              stride is 1, other strides multiples of 8 elements, data 16-byte aligned
+ *   mask_kind  FA_MASK_CAUSAL, or 0 for the plain softmax (the chain's last step alone)
+ *   offset     the position of query row 0 among the keys: row q keeps keys kv <= q + offset
+ *              (K - Q when a chunk of Q queries closes a context of K keys; may be negative)
+ *   probs      (B, H, Q, K), scores' dtype, caller-owned; may be `scores` itself with the same
+ *              strides (each row is read before it is written), otherwise must not overlap it
+ *
+ * Limits: K a multiple of 8 and at most 32768 (else FA_ERR_UNSUPPORTED).  scores and probs
+ * must be memory of the current device.  Asynchronous on `stream`; device-side waits are
+ * bounded, and a wait that runs out sets a status word read by fa_masked_softmax_status.
+ */
+fa_status_t fa_masked_softmax(const fa_tensor_t* scores, uint32_t mask_kind, int64_t offset,
+                              fa_tensor_t* probs, void* stream);
+
+/* Synchronise `stream`, read and clear the status word of the fa_masked_softmax kernels:
+ * FA_OK, FA_ERR_TIMEOUT (a bounded wait ran out), or FA_ERR_CUDA. */
+fa_status_t fa_masked_softmax_status(void* stream);
 
 /* Fill `info` with the mask's extents and device pointers.  FA_ERR_INVALID_ARG on NULL. */
 fa_status_t fa_block_mask_get(const fa_block_mask_t* block_mask, fa_block_mask_info_t* info);
