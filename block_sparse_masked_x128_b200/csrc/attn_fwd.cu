@@ -408,7 +408,8 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                 }
             }
             if (!full) {
-                int lo = 0, hi = kBlock - 1;
+                // Keys past KV_LEN (a ragged last kv tile, zero-filled by TMA) are masked.
+                int lo = 0, hi = min(kBlock - 1, p.KV_LEN - 1 - kv0);
                 if (p.mask_kind & (FA_MASK_CAUSAL | FA_MASK_SLIDING_WINDOW)) hi = min(hi, q - kv0);
                 if (p.mask_kind & FA_MASK_SLIDING_WINDOW) lo = max(lo, q - p.window + 1 - kv0);
                 if constexpr (kDoc) {
@@ -501,6 +502,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
         ++of_cnt;
         tc_fence_after();
         const float inv = (l > 0.f) ? 1.0f / l : 0.f;
+        const bool q_in = q < p.Q_LEN;   // rows past Q_LEN (a ragged last query tile) are not stored
         uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + un.b * p.out_stride[0] +
                          un.h * p.out_stride[1] + (int64_t)q * p.out_stride[2];
 #pragma unroll
@@ -514,11 +516,13 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             for (int i = 0; i < 16; ++i)
                 pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+            if (q_in) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
         }
-        if (p.lse)
+        if (p.lse && q_in)
             p.lse[((int64_t)un.b * p.H + un.h) * p.Q_LEN + q] =
                 (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
         tc_fence_before();

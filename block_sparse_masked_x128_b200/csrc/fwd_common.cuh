@@ -81,8 +81,8 @@ constexpr int kUnitRing = 2;
 
 // Consumer side: the next unit of this CTA, -1 when there is none; ok turns false when the
 // bounded wait gave up.  Called by every lane of a warp.
-template <class C>
-__device__ __forceinline__ int take_unit(const FwdParams& p, uint32_t bars, const volatile int* ring,
+template <class C, class Params>
+__device__ __forceinline__ int take_unit(const Params& p, uint32_t bars, const volatile int* ring,
                                          uint32_t& u_iter, volatile int* abort_flag, bool& ok) {
     const int slot = (int)(u_iter % kUnitRing);
     const uint32_t par = (u_iter / kUnitRing) & 1u;
@@ -208,9 +208,10 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
     finish();
 }
 
-// A query row with no live key: O = 0 and lse = -inf.
+// A query row with no live key: O = 0 and lse = -inf (nothing for rows past Q_LEN).
 template <int D, bool BF16>
 __device__ __forceinline__ void store_row_zero(const FwdParams& p, const Unit& un, int q) {
+    if (q >= p.Q_LEN) return;
     uint16_t* o = reinterpret_cast<uint16_t*>(p.out) + un.b * p.out_stride[0] +
                   un.h * p.out_stride[1] + (int64_t)q * p.out_stride[2];
 #pragma unroll

@@ -163,6 +163,42 @@ def test_query_and_key_lengths_may_differ(Q, KV, kind, window):
     compare(out, lse, O, L)
 
 
+RAGGED = [
+    (1000, 1000, C, 0, 64, "bf16", wl.SCORE_NONE, None),
+    (4097, 4097, C, 0, 128, "bf16", wl.SCORE_NONE, None),
+    (300, 700, C, 0, 128, "fp16", wl.SCORE_NONE, None),
+    (300, 700, C | SW, 100, 64, "fp16", wl.SCORE_NONE, None),
+    (1, 2000, 0, 0, 128, "bf16", wl.SCORE_NONE, None),
+    (17, 333, C, 0, 64, "bf16", wl.SCORE_NONE, None),
+    (1000, 1000, C | DOC, 0, 128, "bf16", wl.SCORE_NONE, [300, 1, 450, 249]),
+    (777, 777, C, 0, 128, "bf16", wl.SCORE_SOFTCAP | wl.SCORE_ALIBI, None),
+]
+
+
+@pytest.mark.parametrize("Q,KV,kind,window,D,dtype,score,doc_lens", RAGGED,
+                         ids=[f"q{r[0]}_kv{r[1]}_m{r[2]}_d{r[4]}_{r[5]}_s{r[6]}" for r in RAGGED])
+def test_ragged_lengths(Q, KV, kind, window, D, dtype, score, doc_lens):
+    # Lengths that are not multiples of 128: the last tile is loaded zero-filled, keys past
+    # KV_LEN are masked and rows past Q_LEN are not stored.
+    w = wl.Workload("ragged", B=2, H=2, S=Q, D=D, dtype=dtype, mask_kind=kind, window=window,
+                    score_kind=score, softcap=30.0, seed=28)
+    fa = fa_module()
+    g = torch.Generator().manual_seed(28 + Q + KV)
+    td = wl.torch_dtype(dtype)
+    q = torch.randn(2, 2, Q, D, generator=g).to(td)
+    k = torch.randn(2, 2, KV, D, generator=g).to(td)
+    v = torch.randn(2, 2, KV, D, generator=g).to(td)
+    doc = wl.doc_ids_from_lengths(doc_lens) if doc_lens else None
+    bm = gpu_block_mask(kind, None, None, Q, KV, window, doc)
+    out = torch.full((2, 2, Q, D), 7.0, dtype=td, device="cuda")   # rows the kernel skips stay 7
+    out, lse = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm, score_mod=score, softcap=30.0,
+                                 out=out)
+    torch.cuda.synchronize()
+    assert bm.device_status() == fa.FA_OK
+    O, L = run_oracle(w, q, k, v, doc)
+    compare(out, lse, O, L)
+
+
 def test_per_head_mask_equals_broadcast_mask():
     fa = fa_module()
     g = torch.Generator().manual_seed(9)
