@@ -104,8 +104,9 @@ def test_forward_rejects_bad_arguments(fa):
     d96 = [_t(fa, D=96) for _ in range(4)]
     assert _fwd(fa, *d96) == fa.FA_ERR_UNSUPPORTED
     assert "head_dim" in fa.fa_last_error_message()
-    r = [_t(fa, S=200) for _ in range(4)]
-    assert _fwd(fa, *r) == fa.FA_ERR_UNSUPPORTED
+    r = [_t(fa, S=200) for _ in range(4)]           # ragged lengths pass the shape checks:
+    assert _fwd(fa, *r) == fa.FA_ERR_INVALID_ARG      # what stops this call is the NULL mask
+    assert "block_mask" in fa.fa_last_error_message()
     assert _fwd(fa, q, k, v, o, kind=4) == fa.FA_ERR_INVALID_ARG                # unknown score bit
     assert _fwd(fa, q, k, v, o, kind=1) == fa.FA_ERR_INVALID_ARG                # soft-cap without params
     assert _fwd(fa, q, k, v, o, kind=1, params=fa.FaScoreParams(0.0, None)) == fa.FA_ERR_INVALID_ARG
@@ -148,11 +149,12 @@ def test_binding_constants_match_the_header(fa):
 
 def test_struct_layouts_match_the_header(fa):
     # ctypes mirrors of the ABI structs: field order and sizes as declared (64-bit ABI).
-    assert ctypes.sizeof(fa.FaMaskParams) == 24      # int32, pad, void*, int32, pad
+    assert ctypes.sizeof(fa.FaMaskParams) == 24      # int32, pad, void*, int32, int32
     assert ctypes.sizeof(fa.FaScoreParams) == 16     # float, pad, const float*
     assert ctypes.sizeof(fa.FaTensor) == 8 + 8 + 4 * 8 + 4 * 8
     text = open(os.path.join(ROOT, "include", "fa_b200.h")).read()
-    for struct, fields in (("fa_mask_params", ["window", "doc_id", "separate_full_blocks"]),
+    for struct, fields in (("fa_mask_params", ["window", "doc_id", "separate_full_blocks",
+                                               "dq_kv_order"]),
                            ("fa_score_params", ["softcap", "alibi_slopes"]),
                            ("fa_tensor", ["data", "dtype", "B", "stride"])):
         body = re.search(r"typedef struct %s \{(.*?)\}" % struct, text, flags=re.S).group(1)
