@@ -51,11 +51,14 @@ def make_score_mod_grad(kind: int, softcap: float = 30.0):
 
 def attention_backward(q, k, v, dout, mask_mod: Callable, score_mod: Optional[Callable] = None,
                        score_mod_grad: Optional[Callable] = None, scale: Optional[float] = None,
-                       chunk: int = 512):
+                       chunk: int = 512, rows=None):
     """(dQ, dK, dV) of sum(dout * O) for O = attention(q, k, v, mask_mod, score_mod, scale).
 
     q: (B, H, Sq, D); k, v: (B, H, Skv, D); dout: (B, H, Sq, D); all upcast to float64.
-    score_mod_grad must be given whenever score_mod is.
+    score_mod_grad must be given whenever score_mod is.  ``rows`` restricts the sum to the
+    given query rows: dQ is then exact on those rows (zero elsewhere) and dK, dV hold those
+    rows' contributions only, which are the whole gradient for any key that no other query
+    row sees (for sampled checks at full size).
     """
     if (score_mod is None) != (score_mod_grad is None):
         raise ValueError("score_mod and score_mod_grad go together")
@@ -66,10 +69,11 @@ def attention_backward(q, k, v, dout, mask_mod: Callable, score_mod: Optional[Ca
         scale = 1.0 / math.sqrt(D)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     kv_idx = np.arange(Skv)[None, :]
+    row_list = np.arange(Sq) if rows is None else np.asarray(rows)
     for b in range(B):
         for h in range(H):
-            for c0 in range(0, Sq, chunk):
-                r = np.arange(c0, min(Sq, c0 + chunk))
+            for c0 in range(0, len(row_list), chunk):
+                r = row_list[c0:c0 + chunk]
                 q_idx = r[:, None]
                 s = scale * (q[b, h, r, :] @ k[b, h].T)
                 s_mod = score_mod(s, b, h, q_idx, kv_idx) if score_mod is not None else s

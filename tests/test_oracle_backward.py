@@ -114,3 +114,20 @@ def test_pin_catches_a_wrong_scale():
     q, k, v, dout = (_rand((1, 1, 6, 3), s) for s in (71, 72, 73, 74))
     grads = oracle.attention_backward(q, k, v, dout, oracle.causal, scale=1.0)
     assert _fd_mismatch(*grads, q, k, v, dout, oracle.causal, None, None) > 1e-3
+
+
+def test_row_subsets_split_the_gradient():
+    # Restricting to query rows R gives exact dQ on R and R's share of dK, dV: two disjoint
+    # subsets add up to the whole, and a key only the last rows see gets its whole gradient
+    # from those rows.
+    g = np.random.default_rng(41)
+    q, k, v, do = (g.standard_normal((1, 2, 40, 8)) for _ in range(4))
+    mm = oracle.causal
+    full = oracle.attention_backward(q, k, v, do, mm)
+    a = oracle.attention_backward(q, k, v, do, mm, rows=np.arange(0, 17))
+    b = oracle.attention_backward(q, k, v, do, mm, rows=np.arange(17, 40))
+    for t in range(3):
+        assert np.abs(a[t] + b[t] - full[t]).max() < 1e-12
+    assert np.array_equal(a[0][:, :, 17:], np.zeros_like(a[0][:, :, 17:]))
+    assert np.abs(b[1][:, :, 17:] - full[1][:, :, 17:]).max() < 1e-12
+    assert np.abs(b[2][:, :, 17:] - full[2][:, :, 17:]).max() < 1e-12

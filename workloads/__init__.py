@@ -105,6 +105,16 @@ def make_qkv(w: Workload, seed: Optional[int] = None):
     return tuple(out)
 
 
+def make_dout(w: Workload, seed: Optional[int] = None):
+    """Upstream gradient dO for the backward: i.i.d. N(0, 1) float32 of shape (B, H, S, D) from
+    ``torch.Generator('cpu').manual_seed(seed + 7919)``, rounded to the workload's dtype."""
+    import torch
+    g = torch.Generator(device="cpu")
+    g.manual_seed((w.seed if seed is None else seed) + 7919)
+    t = torch.randn((w.B, w.H, w.S, w.D), generator=g, dtype=torch.float32)
+    return t.to(torch_dtype(w.dtype))
+
+
 def doc_lengths(total: int, n_docs: int, min_len: int, seed: int) -> list:
     """Seeded document lengths, each >= min_len, summing to total."""
     slack = total - n_docs * min_len
