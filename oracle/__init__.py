@@ -25,7 +25,7 @@ order of soft-cap and ALiBi, for one), the pin checks that reading.
 from .backward import attention_backward, make_score_mod_grad, soft_cap_grad  # noqa: F401
 from .masked_softmax import masked_softmax, causal_keep, finfo_min, BF16_MIN, FP16_MIN  # noqa: F401
 from .attention import (  # noqa: F401
-    causal, sliding_window, document, conjunction, all_true, make_mask_mod,
+    causal, sliding_window, document, sequence_lengths, conjunction, all_true, make_mask_mod,
     dense_mask, soft_cap, alibi, alibi_slopes, compose_score_mods,
     make_score_mod, create_block_mask, attention, live_positions,
     MASK_CAUSAL, MASK_SLIDING_WINDOW, MASK_DOCUMENT, SCORE_SOFTCAP, SCORE_ALIBI,

@@ -55,6 +55,20 @@ def document(document_id):
     return mask_mod
 
 
+def sequence_lengths(kv_lens):
+    """Per-batch context length: key kv_idx of batch b exists iff kv_idx < kv_lens[b].
+
+    A batch of sequences of different lengths shares one KV_LEN-long layout (padded, or paged
+    as PagedAttention through block indices, "PyTorch 2.13 brings custom AI attention to
+    Mac", "What Attention Patterns Does FlexAttention Support?"); the padding is masked.
+    """
+    lens = np.asarray(kv_lens)
+
+    def mask_mod(b, h, q_idx, kv_idx):
+        return kv_idx < lens[b]
+    return mask_mod
+
+
 def all_true(b, h, q_idx, kv_idx):
     """No mask: every pair is allowed."""
     return np.ones(np.broadcast(q_idx, kv_idx).shape, dtype=bool)
@@ -70,9 +84,12 @@ def conjunction(*mods):
     return mask_mod
 
 
-def make_mask_mod(kind: int, window: Optional[int] = None, document_id=None):
-    """The mask_mod for a bit set of kinds (causal 1, sliding window 2, document 4)."""
+def make_mask_mod(kind: int, window: Optional[int] = None, document_id=None, kv_lens=None):
+    """The mask_mod for a bit set of kinds (causal 1, sliding window 2, document 4), AND the
+    per-batch sequence lengths when kv_lens is given."""
     mods = []
+    if kv_lens is not None:
+        mods.append(sequence_lengths(kv_lens))
     if kind & MASK_CAUSAL:
         mods.append(causal)
     if kind & MASK_SLIDING_WINDOW:
@@ -163,11 +180,13 @@ def make_score_mod(kind: int, H: int, softcap: float = 30.0, slopes=None):
 # --------------------------------------------------------------------------
 
 def create_block_mask(mask_mod, B: Optional[int], H: Optional[int], Q_LEN: int,
-                      KV_LEN: int, BLOCK_SIZE: int = 128,
+                      KV_LEN: int, BLOCK_SIZE=128,
                       separate_full_blocks: bool = True) -> dict:
     """Brute-force block metadata from the dense mask.
 
-    The dense mask is reshaped to (QB, BS, KVB, BS) tiles; a tile with no true entry is
+    BLOCK_SIZE is an int or a (q, kv) pair ([CBM] Parameters, BLOCK_SIZE: a single int is used
+    for both query and key/value).  The dense mask is reshaped to (QB, BQ, KVB, BKV) tiles; a
+    tile with no true entry is
     dead (skipped, [FA-Mac] "The two hooks"), a tile whose entries are all true is full,
     and any other live tile is partial.  With separate_full_blocks the full tiles go to
     their own lists so mask_mod can be skipped there; without it every live tile is
@@ -178,9 +197,12 @@ def create_block_mask(mask_mod, B: Optional[int], H: Optional[int], Q_LEN: int,
     indices and is padded with 0 after its count; B or H of None/0 is stored as one
     broadcast entry.
     """
-    BS = int(BLOCK_SIZE)
-    QB = -(-Q_LEN // BS)
-    KVB = -(-KV_LEN // BS)
+    if isinstance(BLOCK_SIZE, (tuple, list)):
+        BQ, BKV = (int(x) for x in BLOCK_SIZE)
+    else:
+        BQ = BKV = int(BLOCK_SIZE)
+    QB = -(-Q_LEN // BQ)
+    KVB = -(-KV_LEN // BKV)
     Bp = 1 if not B else int(B)
     Hp = 1 if not H else int(H)
     kv_num = np.zeros((Bp, Hp, QB), dtype=np.int32)
@@ -190,10 +212,10 @@ def create_block_mask(mask_mod, B: Optional[int], H: Optional[int], Q_LEN: int,
     for b in range(Bp):
         for h in range(Hp):
             for i in range(QB):
-                rows = np.arange(i * BS, min((i + 1) * BS, Q_LEN))
-                m = np.zeros((BS, KVB * BS), dtype=bool)
+                rows = np.arange(i * BQ, min((i + 1) * BQ, Q_LEN))
+                m = np.zeros((BQ, KVB * BKV), dtype=bool)
                 m[: len(rows), :KV_LEN] = dense_mask(mask_mod, Q_LEN, KV_LEN, b, h, rows)
-                tiles = m.reshape(BS, KVB, BS)
+                tiles = m.reshape(BQ, KVB, BKV)
                 any_t = tiles.any(axis=(0, 2))
                 all_t = tiles.all(axis=(0, 2))
                 full = all_t if separate_full_blocks else np.zeros_like(all_t)
@@ -206,7 +228,7 @@ def create_block_mask(mask_mod, B: Optional[int], H: Optional[int], Q_LEN: int,
                 full_idx[b, h, i, : len(f)] = f
     return {"kv_num_blocks": kv_num, "kv_indices": kv_idx,
             "full_kv_num_blocks": full_num, "full_kv_indices": full_idx,
-            "BLOCK_SIZE": BS, "Q_LEN": Q_LEN, "KV_LEN": KV_LEN}
+            "BLOCK_SIZE": (BQ, BKV), "Q_LEN": Q_LEN, "KV_LEN": KV_LEN}
 
 
 def live_positions(mask_mod, Q_LEN: int, KV_LEN: int, b: int = 0, h: int = 0,

@@ -98,16 +98,17 @@ def test_mask_kinds_combine_as_conjunction():
 # ---------------------------------------------------------------- block metadata
 
 def _block_mask_python_loops(pred, Q, KV, BS, separate_full):
-    """Independent brute force: plain loops over tiles and elements."""
-    QB, KVB = -(-Q // BS), -(-KV // BS)
+    """Independent brute force: plain loops over tiles and elements (BS an int or a pair)."""
+    BQ, BKV = BS if isinstance(BS, tuple) else (BS, BS)
+    QB, KVB = -(-Q // BQ), -(-KV // BKV)
     kvn, kvi, fn, fi = [], [], [], []
     for i in range(QB):
         part, full = [], []
         for j in range(KVB):
             n_true, n_all = 0, 0
-            for a in range(BS):
-                for c in range(BS):
-                    qq, kk = i * BS + a, j * BS + c
+            for a in range(BQ):
+                for c in range(BKV):
+                    qq, kk = i * BQ + a, j * BKV + c
                     n_all += 1
                     if qq < Q and kk < KV and pred(qq, kk):
                         n_true += 1
@@ -123,11 +124,11 @@ def _block_mask_python_loops(pred, Q, KV, BS, separate_full):
     return np.array(kvn), np.array(kvi), np.array(fn), np.array(fi)
 
 
+@pytest.mark.parametrize("BS", [4, (4, 3), (2, 5)])
 @pytest.mark.parametrize("separate_full", [True, False])
 @pytest.mark.parametrize("case", ["causal", "swa5", "swa9", "doc", "doc_swa", "none"])
-def test_block_metadata_matches_python_brute_force(case, separate_full):
-    Q = KV = 22           # ragged: not a multiple of BS
-    BS = 4
+def test_block_metadata_matches_python_brute_force(case, separate_full, BS):
+    Q = KV = 22           # ragged: not a multiple of the block sizes
     doc = wl.doc_ids_from_lengths([5, 3, 9, 5])
     preds = {
         "causal": (oracle.MASK_CAUSAL, None, lambda q, k: q >= k),
@@ -463,3 +464,40 @@ def test_pin_catches_a_mask_applied_before_the_soft_cap():
     right = np.where(live, cap * np.tanh(s / cap), -np.inf)
     assert np.abs(np.exp(right - lse[0, 0][:, None]).sum(axis=1) - 1).max() < 1e-12
     assert math.isfinite(float(lse[0, 0, 0]))
+
+
+# ---------------------------------------------------------------- per-batch sequence lengths
+
+def test_sequence_lengths_brute_force():
+    mm = oracle.sequence_lengths([3, 7])
+    for b, L in ((0, 3), (1, 7)):
+        m = oracle.dense_mask(mm, 5, 9, b=b)
+        assert np.array_equal(m, np.array([[kv < L for kv in range(9)] for _ in range(5)]))
+
+
+def test_sequence_lengths_equal_truncated_keys():
+    # A batch element with length L attends exactly as if its K, V had L rows.
+    q, k, v = (_rand((2, 2, 12, 8), s) for s in (61, 62, 63))
+    lens = [5, 12]
+    mm = oracle.make_mask_mod(oracle.MASK_CAUSAL | oracle.MASK_SLIDING_WINDOW, window=4, kv_lens=lens)
+    O, L = oracle.attention(q, k, v, mm)
+    for b, n in enumerate(lens):
+        base = oracle.make_mask_mod(oracle.MASK_CAUSAL | oracle.MASK_SLIDING_WINDOW, window=4)
+        Ob, Lb = oracle.attention(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n], base)
+        assert np.abs(O[b:b + 1] - Ob).max() < 1e-12
+        fin = np.isfinite(Lb)
+        assert np.array_equal(np.isfinite(L[b:b + 1]), fin) and np.abs(L[b:b + 1][fin] - Lb[fin]).max() < 1e-12
+
+
+def test_block_metadata_with_sequence_lengths_is_per_batch():
+    lens = [300, 1000, 129]
+    mm = oracle.make_mask_mod(oracle.MASK_CAUSAL, kv_lens=lens)
+    bm = oracle.create_block_mask(mm, 3, None, 1000, 1000)
+    for b, n in enumerate(lens):
+        one = oracle.create_block_mask(oracle.causal, None, None, 1000, n)
+        kvb = one["kv_indices"].shape[-1]
+        for key in ("kv_num_blocks", "full_kv_num_blocks"):
+            assert np.array_equal(bm[key][b, 0], one[key][0, 0])
+        for key in ("kv_indices", "full_kv_indices"):
+            assert np.array_equal(bm[key][b, 0, :, :kvb], one[key][0, 0])
+            assert np.all(bm[key][b, 0, :, kvb:] == 0)
