@@ -430,6 +430,122 @@ def time_masked_softmax(w: wl.SoftmaxWorkload, steps: int, warmup: int, world: i
             "clocks": clocks.summary()}
 
 
+def time_backward(w: wl.Workload, steps: int, warmup: int, world: int, rank: int, dev) -> dict:
+    """Time fa_backward (pre-pass, dK/dV pass, dQ pass) on one workload, L2 flushed before each
+    step.  Algorithmic FLOPs are 2.5 times the forward's (five 4*D-per-position matmul pairs
+    halved: 10 * D per live position); the kernels execute 14 * D (S and dP are formed in both
+    passes, which keeps every sum on one CTA)."""
+    import torch
+    import block_sparse_masked_x128_b200 as fa
+
+    q, k, v = (t.to(dev) for t in wl.make_qkv(w, seed=rank_plan(w, world, rank)["seed"]))
+    do = wl.make_dout(w, seed=rank_plan(w, world, rank)["seed"]).to(dev)
+    doc = wl.make_doc_ids(w)
+    doc_d = torch.from_numpy(doc).to(dev) if doc is not None else None
+    bm = fa.create_block_mask(w.mask_kind, None, None, w.S, w.S, window=w.window, doc_id=doc_d)
+    out, lse = fa.flex_attention(q, k, v, bm, score_mod=w.score_kind, softcap=w.softcap or 30.0,
+                                 scale=w.scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_backward_workspace_bytes(w.B, w.H, w.S), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def bwd():
+        fa.flex_attention_backward(q, k, v, out, lse, do, bm, score_mod=w.score_kind,
+                                   softcap=w.softcap or 30.0, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                                   workspace=ws)
+
+    for _ in range(warmup):
+        flush.zero_()
+        bwd()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    with ClockSampler(dev.index) as clocks:
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            bwd()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if bm.device_status() != fa.FA_OK:
+        raise RuntimeError("a device-side wait timed out in the backward")
+    per = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    t_max = max_over_ranks(sum(per), world, dev)
+    flops = 2.5 * flops_per_step(w, doc)
+    peaks = read_peaks()
+    achieved = flops / (statistics.mean(per) * 1e-3) / 1e12
+    return {"metric": "live-position attention bwd TFLOP/s (2.5x forward FLOPs)",
+            "value": world * flops * steps / (t_max * 1e-3) / 1e12, "unit": UNIT,
+            "ms_per_step": t_max / steps, "algorithmic_gflop_per_step": flops / 1e9,
+            "executed_gflop_per_step": flops * 1.4 / 1e9, "gpu_launches": 3 * steps,
+            "config": {"workload": w.name, "dtype": w.dtype},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                         "peak_source": peaks["source"] + " bf16_tflops (burst)",
+                         "kernel": "attn_bwd_kernel (dK/dV and dQ passes) + pre-pass"},
+            "clocks": clocks.summary()}
+
+
+def decode_bytes(w: wl.DecodeWorkload) -> int:
+    """Algorithmic bytes of one paged decode step: every live key and value read once (the
+    tokens of each sequence, all heads), q read and out written once, lse written once."""
+    toks = int(w.lengths().astype(np.int64).sum())
+    return int(toks * w.H * w.D * 2 * 2 + 2 * w.B * w.H * w.Q * w.D * 2 + w.B * w.H * w.Q * 4)
+
+
+def time_decode(w: wl.DecodeWorkload, steps: int, warmup: int, world: int, dev) -> dict:
+    """Time one paged decode step (fa_forward_paged over the shuffled page pool), L2 flushed
+    before each step; HBM roofline over the bytes decode_bytes counts."""
+    import torch
+    import block_sparse_masked_x128_b200 as fa
+
+    q, k, v, kp, vp, table, lens = wl.make_decode(w)
+    del k, v
+    q, kp, vp, table = q.to(dev), kp.to(dev), vp.to(dev), table.to(dev)
+    bm = fa.create_block_mask(0, w.B, None, w.Q, w.kv_len, kv_lens=torch.from_numpy(lens).to(dev))
+    out = torch.empty_like(q)
+    lse = torch.empty(w.B, w.H, w.Q, device=dev, dtype=torch.float32)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fa.flex_attention(q, kp, vp, bm, page_table=table, scale=w.scale, out=out, lse=lse)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    with ClockSampler(dev.index) as clocks:
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if bm.device_status() != fa.FA_OK:
+        raise RuntimeError("the paged decode reported a timeout or a page out of range")
+    per = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    t_max = max_over_ranks(sum(per), world, dev)
+    nbytes = decode_bytes(w)
+    peaks = read_peaks()
+    achieved = nbytes / (statistics.mean(per) * 1e-3) / 1e9
+    return {"metric": "paged decode attention GB/s (live K/V read once)",
+            "value": world * nbytes * steps / (t_max * 1e-3) / 1e9, "unit": "GB/s",
+            "ms_per_step": t_max / steps, "bytes_per_step": nbytes, "gpu_launches": steps,
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "D": w.D, "Q": w.Q,
+                       "context_lengths": f"seeded in [{w.lo}, {w.hi}]", "dtype": w.dtype,
+                       "pages": int(sum(-(-int(n) // 128) for n in lens))},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": peaks["source"] + " hbm_gbs", "kernel": "attn_fwd_kernel (paged)"},
+            "clocks": clocks.summary()}
+
+
 def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
     import torch
     import block_sparse_masked_x128_b200 as fa
@@ -553,6 +669,13 @@ def run_ours(args, w: wl.Workload, world: int, rank: int, local: int) -> dict:
             "masked_softmax": time_masked_softmax(wl.SOFTMAX_WORKLOADS[0], args.steps, args.warmup,
                                                   world, dev)}
         torch.cuda.empty_cache()
+        res["next_rows"]["decode_paged"] = time_decode(wl.DECODE_WORKLOADS[0], args.steps,
+                                                       args.warmup, world, dev)
+        torch.cuda.empty_cache()
+        for bw in (wl.WORKLOADS[1], wl.WORKLOADS[4]):
+            res["next_rows"]["backward_" + bw.name] = time_backward(bw, args.steps, args.warmup,
+                                                                     world, rank, dev)
+            torch.cuda.empty_cache()
 
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         q, k, v = wl.make_qkv(w, seed=rank_plan(w, world, rank)["seed"])

@@ -42,12 +42,14 @@ FA_DTYPE_BF16 = 1
 EXPORTED = ("fa_create_block_mask", "fa_forward", "fa_block_mask_get", "fa_get_device_status",
             "fa_destroy_block_mask", "fa_status_string", "fa_last_error_message",
             "fa_create_block_mask_noalloc", "fa_debug_set_stall", "fa_masked_softmax",
-            "fa_masked_softmax_status")
+            "fa_masked_softmax_status", "fa_backward", "fa_backward_workspace_bytes",
+            "fa_block_mask_from_kv_blocks", "fa_forward_paged")
 
 
 class FaMaskParams(ctypes.Structure):
     _fields_ = [("window", ctypes.c_int32), ("doc_id", ctypes.c_void_p),
-                ("separate_full_blocks", ctypes.c_int32), ("dq_kv_order", ctypes.c_int32)]
+                ("separate_full_blocks", ctypes.c_int32), ("dq_kv_order", ctypes.c_int32),
+                ("kv_block_size", ctypes.c_int32), ("kv_lens", ctypes.c_void_p)]
 
 
 class FaScoreParams(ctypes.Structure):
@@ -67,7 +69,10 @@ class FaBlockMaskInfo(ctypes.Structure):
                 ("mask_kind", ctypes.c_uint32), ("window", ctypes.c_int32),
                 ("separate_full_blocks", ctypes.c_int32),
                 ("kv_num_blocks", ctypes.c_void_p), ("kv_indices", ctypes.c_void_p),
-                ("full_kv_num_blocks", ctypes.c_void_p), ("full_kv_indices", ctypes.c_void_p)]
+                ("full_kv_num_blocks", ctypes.c_void_p), ("full_kv_indices", ctypes.c_void_p),
+                ("q_num_blocks", ctypes.c_void_p), ("q_indices", ctypes.c_void_p),
+                ("full_q_num_blocks", ctypes.c_void_p), ("full_q_indices", ctypes.c_void_p),
+                ("dq_kv_order", ctypes.c_int32), ("KV_BLOCK_SIZE", ctypes.c_int32)]
 
 
 _status = ctypes.c_int
@@ -79,6 +84,11 @@ _lib.fa_forward.argtypes = [ctypes.POINTER(FaTensor), ctypes.POINTER(FaTensor), 
                             ctypes.c_void_p, ctypes.c_uint32, ctypes.POINTER(FaScoreParams),
                             ctypes.c_float, ctypes.POINTER(FaTensor), ctypes.c_void_p, ctypes.c_void_p]
 _lib.fa_forward.restype = _status
+_lib.fa_forward_paged.argtypes = [ctypes.POINTER(FaTensor), ctypes.POINTER(FaTensor), ctypes.POINTER(FaTensor),
+                                  ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_uint32,
+                                  ctypes.POINTER(FaScoreParams), ctypes.c_float, ctypes.POINTER(FaTensor),
+                                  ctypes.c_void_p, ctypes.c_void_p]
+_lib.fa_forward_paged.restype = _status
 _lib.fa_create_block_mask_noalloc.argtypes = [
     ctypes.c_uint32, ctypes.POINTER(FaMaskParams), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
     ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -101,6 +111,18 @@ _lib.fa_masked_softmax.argtypes = [ctypes.POINTER(FaTensor), ctypes.c_uint32, ct
 _lib.fa_masked_softmax.restype = _status
 _lib.fa_masked_softmax_status.argtypes = [ctypes.c_void_p]
 _lib.fa_masked_softmax_status.restype = _status
+_lib.fa_block_mask_from_kv_blocks.argtypes = [
+    ctypes.c_uint32, ctypes.POINTER(FaMaskParams), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+    ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+    ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p)]
+_lib.fa_block_mask_from_kv_blocks.restype = _status
+_lib.fa_backward_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
+_lib.fa_backward_workspace_bytes.restype = ctypes.c_size_t
+_lib.fa_backward.argtypes = [ctypes.POINTER(FaTensor)] * 5 + [
+    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint32, ctypes.POINTER(FaScoreParams), ctypes.c_float,
+    ctypes.POINTER(FaTensor), ctypes.POINTER(FaTensor), ctypes.POINTER(FaTensor), ctypes.c_void_p,
+    ctypes.c_size_t, ctypes.c_void_p]
+_lib.fa_backward.restype = _status
 
 
 class FaError(RuntimeError):
@@ -200,6 +222,22 @@ def fa_destroy_block_mask(block_mask: int) -> None:
     _lib.fa_destroy_block_mask(block_mask)
 
 
+def fa_backward_workspace_bytes(B: int, H: int, Q_LEN: int) -> int:
+    return int(_lib.fa_backward_workspace_bytes(B, H, Q_LEN))
+
+
+def fa_backward(q: FaTensor, k: FaTensor, v: FaTensor, out: FaTensor, dout: FaTensor, lse_ptr: int,
+                block_mask: int, score_mod_kind: int, params: Optional[FaScoreParams], scale: float,
+                dq: FaTensor, dk: FaTensor, dv: FaTensor, workspace_ptr: int, workspace_bytes: int,
+                stream=None) -> None:
+    st = _lib.fa_backward(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(out),
+                          ctypes.byref(dout), lse_ptr, block_mask, score_mod_kind,
+                          ctypes.byref(params) if params is not None else None, scale,
+                          ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv), workspace_ptr,
+                          workspace_bytes, _stream_ptr(stream))
+    _check(st, "fa_backward")
+
+
 def fa_masked_softmax(scores: FaTensor, mask_kind: int, offset: int, probs: FaTensor,
                       stream=None) -> None:
     _check(_lib.fa_masked_softmax(ctypes.byref(scores), mask_kind, offset, ctypes.byref(probs),
@@ -263,6 +301,24 @@ class BlockMask:
     def full_kv_indices(self):
         return self._view(self.info.full_kv_indices, self.shape_prefix + (self.info.kv_blocks,))
 
+    @property
+    def q_num_blocks(self):
+        return self._view(self.info.q_num_blocks, (self.info.B, self.info.H, self.info.kv_blocks))
+
+    @property
+    def q_indices(self):
+        return self._view(self.info.q_indices, (self.info.B, self.info.H, self.info.kv_blocks,
+                                                 self.info.q_blocks))
+
+    @property
+    def full_q_num_blocks(self):
+        return self._view(self.info.full_q_num_blocks, (self.info.B, self.info.H, self.info.kv_blocks))
+
+    @property
+    def full_q_indices(self):
+        return self._view(self.info.full_q_indices, (self.info.B, self.info.H, self.info.kv_blocks,
+                                                      self.info.q_blocks))
+
     def device_status(self, stream=None) -> int:
         return fa_get_device_status(self.handle, stream)
 
@@ -288,31 +344,92 @@ def check_doc_id(doc_id, KV_LEN: int, device) -> None:
         raise ValueError(f"doc_id lives on {doc_id.device}, the mask on {device}")
 
 
-def create_block_mask(mask_kind: int, B: Optional[int], H: Optional[int], Q_LEN: int, KV_LEN: int,
-                      *, window: int = 0, doc_id=None, separate_full_blocks: bool = True,
-                      dq_kv_order: bool = True, BLOCK_SIZE: int = 128, device=None,
-                      stream=None) -> BlockMask:
-    """Build a block mask on the current CUDA device (B or H of None broadcasts)."""
+def _block_sizes(BLOCK_SIZE):
+    if isinstance(BLOCK_SIZE, (tuple, list)):
+        bq, bkv = BLOCK_SIZE
+        return int(bq), int(bkv)
+    return int(BLOCK_SIZE), int(BLOCK_SIZE)
+
+
+def _mask_params(mask_kind, KV_LEN, window, doc_id, separate_full_blocks, dq_kv_order, bkv, dev,
+                 kv_lens=None, B=None):
     import torch
-    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     doc_ptr = None
     if doc_id is not None:
         # The C ABI reads KV_LEN ids through a bare pointer: check what it cannot.
         check_doc_id(doc_id, KV_LEN, dev)
         doc_ptr = doc_id.data_ptr()
-    params = FaMaskParams(int(window), doc_ptr, 1 if separate_full_blocks else 0,
-                          1 if dq_kv_order else 0)
+    lens_ptr = None
+    if kv_lens is not None:
+        # ... and B context lengths, one per batch element.
+        if not (kv_lens.is_cuda and kv_lens.dtype == torch.int32 and kv_lens.is_contiguous()
+                and kv_lens.dim() == 1 and B and kv_lens.numel() == int(B)
+                and kv_lens.device == torch.device(dev)):
+            raise ValueError("kv_lens must be a contiguous int32 CUDA tensor of B lengths on the "
+                             "mask's device (and B must be given)")
+        lens_ptr = kv_lens.data_ptr()
+    return FaMaskParams(int(window), doc_ptr, 1 if separate_full_blocks else 0,
+                        1 if dq_kv_order else 0, int(bkv), lens_ptr)
+
+
+def create_block_mask(mask_kind: int, B: Optional[int], H: Optional[int], Q_LEN: int, KV_LEN: int,
+                      *, window: int = 0, doc_id=None, separate_full_blocks: bool = True,
+                      dq_kv_order: bool = True, BLOCK_SIZE=128, kv_lens=None, device=None,
+                      stream=None) -> BlockMask:
+    """Build a block mask on the current CUDA device (B or H of None broadcasts).
+    BLOCK_SIZE is an int or a (q, kv) pair: the block size of the lists read back.  kv_lens
+    (int32 CUDA tensor of B lengths) masks keys past each batch element's context."""
+    import torch
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    bq, bkv = _block_sizes(BLOCK_SIZE)
+    params = _mask_params(mask_kind, KV_LEN, window, doc_id, separate_full_blocks, dq_kv_order, bkv, dev,
+                          kv_lens, B)
     with torch.cuda.device(dev):
         h = fa_create_block_mask(int(mask_kind), params, int(B or 0), int(H or 0), int(Q_LEN),
-                                 int(KV_LEN), int(BLOCK_SIZE), stream)
-    # doc_id is copied on the stream; keep it alive until the caller's stream has run it.
-    return BlockMask(h, dev, keepalive=doc_id)
+                                 int(KV_LEN), bq, stream)
+    # doc_id and kv_lens are copied on the stream; keep them alive until the stream has run.
+    return BlockMask(h, dev, keepalive=(doc_id, kv_lens))
+
+
+def block_mask_from_kv_blocks(kv_num_blocks, kv_indices, full_kv_num_blocks=None,
+                              full_kv_indices=None, *, Q_LEN: int, KV_LEN: int, BLOCK_SIZE=128,
+                              mask_kind: int = 0, window: int = 0, doc_id=None,
+                              separate_full_blocks: bool = True, dq_kv_order: bool = True,
+                              stream=None) -> BlockMask:
+    """BlockMask.from_kv_blocks: a mask from caller block lists (int32 CUDA tensors of shape
+    (B, H, QBu) and (B, H, QBu, KVBu)); block sizes must be multiples of 128.  mask_kind and
+    its parameters give the mask_mod applied on partial blocks (0: none)."""
+    import torch
+    bq, bkv = _block_sizes(BLOCK_SIZE)
+    dev = kv_indices.device
+    B, H = kv_indices.shape[0], kv_indices.shape[1]
+    lists = [kv_num_blocks, kv_indices] + ([full_kv_num_blocks, full_kv_indices]
+                                           if full_kv_num_blocks is not None else [])
+    QBu, KVBu = -(-int(Q_LEN) // bq), -(-int(KV_LEN) // bkv)
+    for t, shape in zip(lists, [(B, H, QBu), (B, H, QBu, KVBu)] * 2):
+        if not (t.is_cuda and t.dtype == torch.int32 and t.is_contiguous() and tuple(t.shape) == shape
+                and t.device == dev):
+            raise ValueError(f"block lists must be contiguous int32 CUDA tensors of shape {shape}")
+    params = _mask_params(mask_kind, KV_LEN, window, doc_id, separate_full_blocks, dq_kv_order, bkv, dev)
+    h = ctypes.c_void_p()
+    with torch.cuda.device(dev):
+        st = _lib.fa_block_mask_from_kv_blocks(
+            int(mask_kind), ctypes.byref(params), B, H, int(Q_LEN), int(KV_LEN), bq, bkv,
+            kv_num_blocks.data_ptr(), kv_indices.data_ptr(),
+            full_kv_num_blocks.data_ptr() if full_kv_num_blocks is not None else None,
+            full_kv_indices.data_ptr() if full_kv_indices is not None else None,
+            _stream_ptr(stream), ctypes.byref(h))
+    _check(st, "fa_block_mask_from_kv_blocks")
+    return BlockMask(h.value, dev, keepalive=(doc_id, lists))
 
 
 def flex_attention(q, k, v, block_mask: BlockMask, *, score_mod: int = FA_SCORE_NONE,
                    softcap: float = 30.0, alibi_slopes=None, scale: Optional[float] = None,
-                   out=None, lse=None, return_lse: bool = True, stream=None) -> Tuple:
-    """Fused block-sparse attention forward: returns (out, lse) (lse None if not requested)."""
+                   out=None, lse=None, return_lse: bool = True, page_table=None,
+                   stream=None) -> Tuple:
+    """Fused block-sparse attention forward: returns (out, lse) (lse None if not requested).
+    With page_table (int32 CUDA tensor (B, n) of page indices), k and v are (n_pages, H, 128, D)
+    page pools and the mask's KV_LEN is the logical context length."""
     import torch
     if out is None:
         out = torch.empty_like(q)
@@ -324,22 +441,70 @@ def flex_attention(q, k, v, block_mask: BlockMask, *, score_mod: int = FA_SCORE_
                 and tuple(lse.shape) == tuple(q.shape[:3]) and lse.device == q.device):
             raise ValueError("lse must be a contiguous float32 CUDA tensor of shape (B, H, Q_LEN) "
                              "on q's device")
-    slopes_ptr = None
-    if alibi_slopes is not None:
-        # The kernel reads slope h for h < H through a bare pointer: H contiguous floats.
-        if not (alibi_slopes.is_cuda and alibi_slopes.dtype == torch.float32
-                and alibi_slopes.is_contiguous() and alibi_slopes.numel() == q.shape[1]
-                and alibi_slopes.device == q.device):
-            raise ValueError("alibi_slopes must be a contiguous float32 CUDA tensor of H "
-                             "values on q's device")
-        slopes_ptr = alibi_slopes.data_ptr()
-    params = FaScoreParams(float(softcap), slopes_ptr)
+    params = FaScoreParams(float(softcap), _check_alibi(alibi_slopes, q))
     with torch.cuda.device(q.device if q.is_cuda else block_mask.device):
-        fa_forward(fa_tensor(q), fa_tensor(k), fa_tensor(v), block_mask.handle, int(score_mod), params,
-                   float(scale) if scale is not None else -1.0, fa_tensor(out),
-                   lse.data_ptr() if lse is not None else None, stream)
+        if page_table is None:
+            fa_forward(fa_tensor(q), fa_tensor(k), fa_tensor(v), block_mask.handle, int(score_mod), params,
+                       float(scale) if scale is not None else -1.0, fa_tensor(out),
+                       lse.data_ptr() if lse is not None else None, stream)
+        else:
+            # The C ABI reads the table through a bare pointer: rows of kv_blocks entries.
+            if not (page_table.is_cuda and page_table.dtype == torch.int32 and page_table.dim() == 2
+                    and page_table.stride(1) == 1 and page_table.shape[0] == q.shape[0]
+                    and page_table.shape[1] >= -(-block_mask.info.KV_LEN // 128)
+                    and page_table.device == q.device):
+                raise ValueError("page_table must be an int32 CUDA tensor (B, >= kv blocks) with "
+                                 "contiguous rows on q's device")
+            st = _lib.fa_forward_paged(ctypes.byref(fa_tensor(q)), ctypes.byref(fa_tensor(k)),
+                                       ctypes.byref(fa_tensor(v)), page_table.data_ptr(),
+                                       page_table.stride(0), block_mask.handle, int(score_mod),
+                                       ctypes.byref(params), float(scale) if scale is not None else -1.0,
+                                       ctypes.byref(fa_tensor(out)),
+                                       lse.data_ptr() if lse is not None else None, _stream_ptr(stream))
+            _check(st, "fa_forward_paged")
     return out, lse
 
+
+
+def _check_alibi(alibi_slopes, q):
+    if alibi_slopes is None:
+        return None
+    import torch
+    # The kernels read slope h for h < H through a bare pointer: H contiguous floats.
+    if not (alibi_slopes.is_cuda and alibi_slopes.dtype == torch.float32
+            and alibi_slopes.is_contiguous() and alibi_slopes.numel() == q.shape[1]
+            and alibi_slopes.device == q.device):
+        raise ValueError("alibi_slopes must be a contiguous float32 CUDA tensor of H "
+                         "values on q's device")
+    return alibi_slopes.data_ptr()
+
+
+def flex_attention_backward(q, k, v, out, lse, dout, block_mask: BlockMask, *,
+                            score_mod: int = FA_SCORE_NONE, softcap: float = 30.0, alibi_slopes=None,
+                            scale: Optional[float] = None, dq=None, dk=None, dv=None,
+                            workspace=None, stream=None) -> Tuple:
+    """Gradients (dq, dk, dv) of flex_attention for the upstream gradient dout, given the
+    forward's out and lse; deterministic (bitwise repeatable)."""
+    import torch
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous()
+            and tuple(lse.shape) == tuple(q.shape[:3]) and lse.device == q.device):
+        raise ValueError("lse must be the forward's contiguous float32 (B, H, Q_LEN) CUDA tensor")
+    nbytes = fa_backward_workspace_bytes(q.shape[0], q.shape[1], q.shape[2])
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() * workspace.element_size() < nbytes or not workspace.is_cuda:
+        raise ValueError(f"workspace must be a CUDA buffer of at least {nbytes} bytes")
+    params = FaScoreParams(float(softcap), _check_alibi(alibi_slopes, q))
+    with torch.cuda.device(q.device):
+        fa_backward(fa_tensor(q), fa_tensor(k), fa_tensor(v), fa_tensor(out), fa_tensor(dout),
+                    lse.data_ptr(), block_mask.handle, int(score_mod), params,
+                    float(scale) if scale is not None else -1.0, fa_tensor(dq), fa_tensor(dk),
+                    fa_tensor(dv), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                    stream)
+    return dq, dk, dv
 
 
 def masked_softmax(scores, offset: Optional[int] = None, *, causal: bool = True, out=None,

@@ -333,6 +333,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             continue;
         }
         const int q = qblk * kBlock + row;
+        const int kv_len = p.kv_lens ? min(p.KV_LEN, __ldg(p.kv_lens + un.b)) : p.KV_LEN;
         float slope_log2 = 0.f;
         if constexpr (has_alibi) {
             float slope;
@@ -408,8 +409,9 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                 }
             }
             if (!full) {
-                // Keys past KV_LEN (a ragged last kv tile, zero-filled by TMA) are masked.
-                int lo = 0, hi = min(kBlock - 1, p.KV_LEN - 1 - kv0);
+                // Keys past the context (a ragged last kv tile, zero-filled by TMA, or this
+                // batch's own length) are masked.
+                int lo = 0, hi = min(kBlock - 1, kv_len - 1 - kv0);
                 if (p.mask_kind & (FA_MASK_CAUSAL | FA_MASK_SLIDING_WINDOW)) hi = min(hi, q - kv0);
                 if (p.mask_kind & FA_MASK_SLIDING_WINDOW) lo = max(lo, q - p.window + 1 - kv0);
                 if constexpr (kDoc) {

@@ -24,13 +24,18 @@ constexpr int kDead = 0, kPartial = 1, kFull = 2, kAmbiguous = 3;
 // query tiles of a work unit (query blocks 2p and 2p+1).
 constexpr int kLive0 = 1 << 16, kFull0 = 1 << 17, kLive1 = 1 << 18, kFull1 = 1 << 19;
 
-// Inputs of the mask-builder kernels.
+// Inputs of the mask-builder kernels.  Tiles are BQ query rows by BKV keys (128 x 128 for the
+// lists the attention kernels walk; a caller's BLOCK_SIZE for the lists it reads back).
 struct MaskSpec {
     uint32_t kind;
     int32_t window;
     int32_t Q_LEN, KV_LEN, QB, KVB;
-    const int32_t* doc;        // [KV_LEN] or null
-    const int32_t* doc_stats;  // [max(QB,KVB)][3] = {min, max, uniform} per block, or null
+    int32_t BQ, BKV;
+    const int32_t* doc;           // [KV_LEN] or null
+    const int32_t* doc_stats;     // [QB][3] = {min, max, uniform} per query block, or null
+    const int32_t* doc_stats_kv;  // [KVB][3] per kv block (== doc_stats when BQ == BKV)
+    const int32_t* kv_lens;       // [B] per-batch context lengths, or null
+    int32_t maskH;                // stored H (row bh of the lists is batch bh / maskH)
 };
 
 // Kernel parameters of the fused forward (passed by value, __grid_constant__).
@@ -39,10 +44,15 @@ struct FwdParams {
     int32_t QB, KVB, NP;          // query blocks, kv blocks, work-unit pairs per (b, h)
     int32_t maskB, maskH;         // stored mask extents (1 = broadcast)
     int32_t n_units;              // NP * B * H
+    int32_t head_major;           // 1: the units of one (b, h) are handed out together
     uint32_t mask_kind;
     int32_t window;
     uint32_t score_kind;
     const int32_t* doc_id;
+    const int32_t* kv_lens;       // [B] per-batch context lengths, or null (all KV_LEN)
+    const int32_t* page_table;    // [B][page_stride] physical page of each kv block, or null
+    int32_t page_stride;
+    int32_t n_pages;              // pages in the K/V pools (the pools' batch extent)
     const int32_t* sched_order;   // [maskB*maskH][NP]  pairs by descending cost
     const int32_t* sched_count;   // [maskB*maskH][NP][2]  entries; live tiles t0 | t1 << 16
     const int32_t* sched_entries; // [maskB*maskH][NP][KVB]
@@ -92,6 +102,7 @@ struct BwdParams {
     int32_t window;
     uint32_t score_kind;
     const int32_t* doc_id;
+    const int32_t* kv_lens;       // [B] per-batch context lengths, or null (all KV_LEN)
     const int32_t* order;         // [maskB*maskH][units_per_bh]  units by descending cost
     const int32_t* count;         // [maskB*maskH][units_per_bh]  entries per unit
     const int32_t* entries;       // [maskB*maskH][units_per_bh][entries_stride]
@@ -121,6 +132,22 @@ cudaError_t launch_attn_bwd_dkdv(const BwdParams& p, int D, bool bf16, int score
 cudaError_t launch_attn_bwd_dq(const BwdParams& p, int D, bool bf16, int score_kind,
                                const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                const CUtensorMap& tdo, int grid, cudaStream_t stream);
+
+cudaError_t launch_expand_block_lists(int UQB, int UKVB, int rq, int rkv, int QB, int KVB, int Q_LEN,
+                                      int KV_LEN, const int32_t* kv_lens, int maskH, int maskBH,
+                                      int separate_full,
+                                      const int32_t* u_kv_num, const int32_t* u_kv_idx,
+                                      const int32_t* u_full_num, const int32_t* u_full_idx,
+                                      int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
+                                      int32_t* full_idx, int32_t* bad, cudaStream_t stream);
+cudaError_t launch_transpose_lists(int QB, int KVB, int maskBH, const int32_t* kv_num,
+                                   const int32_t* kv_idx, const int32_t* full_num,
+                                   const int32_t* full_idx, int32_t* q_num, int32_t* q_idx,
+                                   int32_t* fq_num, int32_t* fq_idx, cudaStream_t stream);
+cudaError_t launch_schedule(int QB, int KVB, int maskBH, int NP, const int32_t* kv_num,
+                            const int32_t* kv_idx, const int32_t* full_num, const int32_t* full_idx,
+                            int32_t* sched_count, int32_t* sched_cost, int32_t* sched_entries,
+                            int32_t* sched_order, cudaStream_t stream);
 
 cudaError_t launch_mask_build(const MaskSpec& spec, int separate_full, int maskBH, int NP,
                               int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
@@ -171,11 +198,18 @@ struct fa_block_mask {
     int32_t* full_idx;
     int32_t* doc;
     int32_t* doc_stats;
+    int32_t* kv_lens;         // copy of the per-batch context lengths, or null
     int32_t* sched_count;
     int32_t* sched_cost;
     int32_t* sched_entries;
     int32_t* sched_order;
     int32_t* status;
+    // The lists a caller reads back (fa_block_mask_get), at its block size BQ x BKV: the
+    // kernel's own 128 x 128 lists when that is the block size, separate arrays otherwise.
+    int32_t BQ, BKV, UQB, UKVB;
+    int32_t *u_kv_num, *u_kv_idx, *u_full_num, *u_full_idx;
+    int32_t *u_q_num, *u_q_idx, *u_fq_num, *u_fq_idx;
+    int32_t* u_doc_stats;
     int32_t dq_kv_order;      // 1: dQ accumulates kv blocks in descending order, 0: ascending
     fa::BwdMeta bwd;
     int32_t* sched_ctr;       // fa::kSchedCtrSlots pairs of unit counters after the status word

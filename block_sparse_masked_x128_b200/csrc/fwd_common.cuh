@@ -32,9 +32,20 @@ struct Unit {
     const int32_t* entries;
 };
 
+// Units are ranked per (b, h) by descending cost.  Interleaved order (the r-th longest unit of
+// every (b, h), then the (r+1)-th ...) hands the longest units of the whole job out first;
+// head-major order keeps the CTAs in flight on one or two (b, h) at a time, so their K and V
+// stay in L2 when all heads' K and V together would not fit.
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     const int BH = p.B * p.H;
-    const int r = u / BH, bh = u - r * BH;
+    int r, bh;
+    if (p.head_major) {
+        bh = u / p.NP;
+        r = u - bh * p.NP;
+    } else {
+        r = u / BH;
+        bh = u - r * BH;
+    }
     const int b = bh / p.H, h = bh - b * p.H;
     const int mb = (p.maskB == 1) ? 0 : b, mh = (p.maskH == 1) ? 0 : h;
     const size_t sidx = (size_t)mb * p.maskH + mh;
@@ -181,6 +192,17 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
         er.init(un.entries, un.E);
         for (int e = 0; e < un.E && ok; ++e) {
             const int j = er.get(e) & 0xFFFF;
+            // K_j and V_j: rows j*128.. of batch b, or with paged K/V the page the table gives
+            // for (b, j) (a page outside the pools is recorded and reads as zeros).
+            int kv_row = j * kBlock, kv_batch = un.b;
+            if (p.page_table) {
+                int page = 0;
+                if (leader) page = __ldg(p.page_table + (size_t)un.b * p.page_stride + j);
+                page = __shfl_sync(kFullMask, page, leader_lane);
+                if (leader && (page < 0 || page >= p.n_pages)) atomicExch(p.status, 2);
+                kv_row = 0;
+                kv_batch = page;
+            }
             for (int which = 0; which < 2; ++which) {
                 const int s = (int)(kv_pos % C::kStages);
                 const uint32_t ph = (kv_pos / C::kStages) & 1u;
@@ -191,7 +213,7 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
                 const CUtensorMap* tm = which ? tmv : tmk;
                 for (int c = 0; c < C::kChunks; ++c)
                     tma_load_4d_if(leader, sKV + s * C::kTileBytes + c * 16384, tm,
-                                   bar(C::kBarSlotFull + s), c * 64, j * kBlock, un.h, un.b);
+                                   bar(C::kBarSlotFull + s), c * 64, kv_row, un.h, kv_batch);
                 ++kv_pos;
             }
         }

@@ -33,12 +33,12 @@ namespace {
 constexpr int kThreads = 128;  // == kBlock: one thread per query row when resolving a tile
 
 __global__ void __launch_bounds__(kThreads) doc_block_stats_kernel(const int32_t* __restrict__ doc,
-                                                                  int len, int nblk,
+                                                                  int len, int nblk, int bs,
                                                                   int32_t* __restrict__ stats) {
     const int blk = blockIdx.x;
     if (blk >= nblk) return;
-    const int s0 = blk * kBlock;
-    const int n = min(kBlock, len - s0);
+    const int s0 = blk * bs;
+    const int n = min(bs, len - s0);
     int mn = INT_MAX, mx = INT_MIN;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int d = doc[s0 + i];
@@ -76,9 +76,9 @@ __device__ __forceinline__ void interval_bounds(const MaskSpec& m, long long& lo
 }
 
 __device__ int classify_fast(const MaskSpec& m, int i, int j) {
-    const int qs = i * kBlock, qe = min(qs + kBlock, m.Q_LEN) - 1;
-    const int ks = j * kBlock, ke = min(ks + kBlock, m.KV_LEN) - 1;
-    const bool ragged = (qe - qs + 1 < kBlock) || (ke - ks + 1 < kBlock);
+    const int qs = i * m.BQ, qe = min(qs + m.BQ, m.Q_LEN) - 1;
+    const int ks = j * m.BKV, ke = min(ks + m.BKV, m.KV_LEN) - 1;
+    const bool ragged = (qe - qs + 1 < m.BQ) || (ke - ks + 1 < m.BKV);
     long long lo, hi;
     interval_bounds(m, lo, hi);
     const long long dmin = (long long)qs - ke, dmax = (long long)qe - ks;
@@ -86,7 +86,7 @@ __device__ int classify_fast(const MaskSpec& m, int i, int j) {
     const bool interval_full = dmin >= lo && dmax <= hi;
     if (!(m.kind & FA_MASK_DOCUMENT)) return (interval_full && !ragged) ? kFull : kPartial;
     const int32_t* qst = m.doc_stats + 3 * i;
-    const int32_t* kst = m.doc_stats + 3 * j;
+    const int32_t* kst = m.doc_stats_kv + 3 * j;
     if (qst[1] < kst[0] || kst[1] < qst[0]) return kDead;   // id ranges disjoint
     if (qst[2] && kst[2]) {                                  // both blocks hold one id
         if (qst[0] != kst[0]) return kDead;
@@ -95,27 +95,39 @@ __device__ int classify_fast(const MaskSpec& m, int i, int j) {
     return kAmbiguous;
 }
 
-// Element-by-element classification of one tile by the whole CTA (thread r = query row r).
-__device__ int resolve_tile(const MaskSpec& m, int i, int j) {
+// Element-by-element classification of one tile by one warp: lane l walks query rows l,
+// l + 32, ... across the tile's keys; the warp stops as soon as it has seen both an allowed
+// and a masked pair (a partial tile), so only dead and full tiles are read in full.
+__device__ int resolve_tile_warp(const MaskSpec& m, int i, int j) {
     long long lo, hi;
     interval_bounds(m, lo, hi);
-    const int q = i * kBlock + threadIdx.x;
-    const bool q_in = q < m.Q_LEN;
-    const int dq = (q_in && m.doc) ? m.doc[q] : 0;
+    const int lane = threadIdx.x & 31;
+    const int q0 = i * m.BQ, k0 = j * m.BKV;
     bool any = false, all = true;
-    for (int c = 0; c < kBlock; ++c) {
-        const int kv = j * kBlock + c;
-        bool live = q_in && kv < m.KV_LEN;
-        if (live) {
-            const long long d = (long long)q - kv;
-            live = d >= lo && d <= hi;
-            if (live && (m.kind & FA_MASK_DOCUMENT)) live = (m.doc[kv] == dq);
+    for (int rb = 0; rb < m.BQ; rb += 32) {
+        const int q = q0 + rb + lane;
+        const bool q_row = rb + lane < m.BQ;
+        if (q_row) {
+            const bool q_in = q < m.Q_LEN;
+            const int dq = (q_in && m.doc) ? m.doc[q] : 0;
+            for (int c = 0; c < m.BKV; ++c) {
+                const int kv = k0 + c;
+                bool live = q_in && kv < m.KV_LEN;
+                if (live) {
+                    const long long d = (long long)q - kv;
+                    live = d >= lo && d <= hi;
+                    if (live && (m.kind & FA_MASK_DOCUMENT)) live = (m.doc[kv] == dq);
+                }
+                any |= live;
+                all &= live;
+            }
         }
-        any |= live;
-        all &= live;
+        const bool a = __any_sync(0xffffffffu, any);
+        const bool f = __all_sync(0xffffffffu, all);
+        if (a && !f) return kPartial;
     }
-    const int a = __syncthreads_or(any ? 1 : 0);
-    const int f = __syncthreads_and(all ? 1 : 0);
+    const bool a = __any_sync(0xffffffffu, any);
+    const bool f = __all_sync(0xffffffffu, all);
     return !a ? kDead : (f ? kFull : kPartial);
 }
 
@@ -125,6 +137,8 @@ classify_compact_kernel(MaskSpec m, int separate_full, int32_t* __restrict__ kv_
                         int32_t* __restrict__ full_idx) {
     const int i = blockIdx.x;
     const int bh = blockIdx.y;
+    // Per-batch context length: keys past it count as masked (the block grid stays KVB wide).
+    if (m.kv_lens) m.KV_LEN = max(0, min(m.KV_LEN, m.kv_lens[bh / m.maskH]));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     __shared__ int s_cls[kThreads];
     __shared__ int s_amb[kThreads];
@@ -144,10 +158,10 @@ classify_compact_kernel(MaskSpec m, int separate_full, int32_t* __restrict__ kv_
         s_cls[tid] = cls;
         __syncthreads();
         const int namb = s_namb;
-        for (int a = 0; a < namb; ++a) {
+        for (int a = warp; a < namb; a += kThreads / 32) {   // one warp per ambiguous tile
             const int t = s_amb[a];
-            const int c = resolve_tile(m, i, jb + t);
-            if (tid == 0) s_cls[t] = c;
+            const int c = resolve_tile_warp(m, i, jb + t);
+            if (lane == 0) s_cls[t] = c;
         }
         __syncthreads();
         cls = s_cls[tid];
@@ -265,20 +279,305 @@ __global__ void __launch_bounds__(1024) lpt_order_kernel(int NP, const int32_t* 
     }
 }
 
+// ------------------------------------------------------------------ backward metadata
+
+__device__ __forceinline__ bool sorted_contains(const int32_t* __restrict__ a, int n, int x) {
+    int lo = 0, hi = n - 1;
+    while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        const int v = a[mid];
+        if (v == x) return true;
+        if (v < x) lo = mid + 1; else hi = mid - 1;
+    }
+    return false;
+}
+
+// Transposed lists (per kv block, the query blocks whose tile is partial / full, ascending)
+// and the kv-major entries of the dK/dV kernel: query block i | kLive0 (| kFull0), ascending.
+// One CTA per (stored b/h, kv block); each thread looks its query row's tile up in the row's
+// sorted lists.
+__global__ void __launch_bounds__(kThreads)
+transpose_lists_kernel(int QB, int KVB, const int32_t* __restrict__ kv_num,
+                       const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ full_num,
+                       const int32_t* __restrict__ full_idx, int32_t* __restrict__ q_num,
+                       int32_t* __restrict__ q_idx, int32_t* __restrict__ fq_num,
+                       int32_t* __restrict__ fq_idx, int32_t* __restrict__ kv_count,
+                       int32_t* __restrict__ kv_cost, int32_t* __restrict__ kv_entries) {
+    const int j = blockIdx.x, bh = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int s_wp[kThreads / 32], s_wf[kThreads / 32];
+    const size_t col = (size_t)bh * KVB + j;
+    int32_t* my_q = q_idx + col * QB;
+    int32_t* my_fq = fq_idx + col * QB;
+    int32_t* my_e = kv_entries ? kv_entries + col * QB : nullptr;
+    int np = 0, nf = 0;
+    for (int ib = 0; ib < QB; ib += kThreads) {
+        const int i = ib + tid;
+        int cls = kDead;
+        if (i < QB) {
+            const size_t row = (size_t)bh * QB + i;
+            const int n_p = min(max(kv_num[row], 0), KVB), n_f = min(max(full_num[row], 0), KVB);
+            if (sorted_contains(full_idx + row * KVB, n_f, j)) cls = kFull;
+            else if (sorted_contains(kv_idx + row * KVB, n_p, j)) cls = kPartial;
+        }
+        const unsigned bp = __ballot_sync(0xffffffffu, cls == kPartial);
+        const unsigned bf = __ballot_sync(0xffffffffu, cls == kFull);
+        if (lane == 0) {
+            s_wp[warp] = __popc(bp);
+            s_wf[warp] = __popc(bf);
+        }
+        __syncthreads();
+        int op = np, of = nf, tp = 0, tf = 0;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            if (w < warp) {
+                op += s_wp[w];
+                of += s_wf[w];
+            }
+            tp += s_wp[w];
+            tf += s_wf[w];
+        }
+        const unsigned lt = (1u << lane) - 1u;
+        if (cls == kPartial) my_q[op + __popc(bp & lt)] = i;
+        if (cls == kFull) my_fq[of + __popc(bf & lt)] = i;
+        // Merged entries in ascending i: the live tiles before this thread's come first.
+        const unsigned bl = bp | bf;
+        if (cls != kDead && kv_entries)
+            my_e[op + of + __popc(bl & lt)] =
+                i | kLive0 | (cls == kFull ? kFull0 : 0);
+        np += tp;
+        nf += tf;
+        __syncthreads();
+    }
+    for (int t = np + tid; t < QB; t += kThreads) my_q[t] = 0;
+    for (int t = nf + tid; t < QB; t += kThreads) my_fq[t] = 0;
+    if (kv_entries)
+        for (int t = np + nf + tid; t < QB; t += kThreads) my_e[t] = 0;
+    if (tid == 0) {
+        q_num[col] = np;
+        fq_num[col] = nf;
+        if (kv_count) {
+            kv_count[col] = np + nf;
+            kv_cost[col] = np + nf + 1;
+        }
+    }
+}
+
+// Per query block, the merged kv list (partial | full) of the dQ kernel: kv block j | kLive0
+// (| kFull0), in descending j when `descending`, else ascending.  This is the order in which
+// the block's dQ accumulates its kv contributions (the dQ write order), fixed per mask.
+__global__ void __launch_bounds__(kThreads)
+dq_entries_kernel(int QB, int KVB, int descending, const int32_t* __restrict__ kv_num,
+                  const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ full_num,
+                  const int32_t* __restrict__ full_idx, int32_t* __restrict__ dq_count,
+                  int32_t* __restrict__ dq_cost, int32_t* __restrict__ dq_entries) {
+    extern __shared__ uint8_t s_code[];
+    const int i = blockIdx.x, bh = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int s_w[kThreads / 32];
+    const size_t row = (size_t)bh * QB + i;
+    for (int j = tid; j < KVB; j += kThreads) s_code[j] = 0;
+    __syncthreads();
+    const int n_p = min(max(kv_num[row], 0), KVB), n_f = min(max(full_num[row], 0), KVB);
+    for (int n = tid; n < n_p; n += kThreads) {
+        const int j = kv_idx[row * KVB + n];
+        if (j >= 0 && j < KVB) s_code[j] = 1;
+    }
+    for (int n = tid; n < n_f; n += kThreads) {
+        const int j = full_idx[row * KVB + n];
+        if (j >= 0 && j < KVB) s_code[j] = 3;
+    }
+    __syncthreads();
+    int32_t* out = dq_entries + row * KVB;
+    int cnt = 0;
+    for (int jb = 0; jb < KVB; jb += kThreads) {
+        const int t = jb + tid;
+        const int j = descending ? KVB - 1 - t : t;
+        const int c = (t < KVB) ? s_code[j] : 0;
+        const unsigned b = __ballot_sync(0xffffffffu, c != 0);
+        if (lane == 0) s_w[warp] = __popc(b);
+        __syncthreads();
+        int off = cnt, tot = 0;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            if (w < warp) off += s_w[w];
+            tot += s_w[w];
+        }
+        if (c != 0) out[off + __popc(b & ((1u << lane) - 1u))] = j | kLive0 | (c == 3 ? kFull0 : 0);
+        cnt += tot;
+        __syncthreads();
+    }
+    for (int t = cnt + tid; t < KVB; t += kThreads) out[t] = 0;
+    if (tid == 0) {
+        dq_count[row] = cnt;
+        dq_cost[row] = cnt + 1;
+    }
+}
+
+// Lists of 128 x 128 tiles from caller lists of BQ x BKV blocks (BQ = rq * 128,
+// BKV = rkv * 128): each tile takes its block's class (a block listed as both partial and full
+// counts as partial), a ragged tile is never full, and an index outside the block grid or a
+// count outside [0, UKVB] sets *bad and is ignored.  One CTA per (stored b/h, query tile).
+__global__ void __launch_bounds__(kThreads)
+expand_block_lists_kernel(int UQB, int UKVB, int rq, int rkv, int QB, int KVB, int Q_LEN, int KV_LEN,
+                          const int32_t* __restrict__ kv_lens, int maskH,
+                          int separate_full, const int32_t* __restrict__ u_kv_num,
+                          const int32_t* __restrict__ u_kv_idx, const int32_t* __restrict__ u_full_num,
+                          const int32_t* __restrict__ u_full_idx, int32_t* __restrict__ kv_num,
+                          int32_t* __restrict__ kv_idx, int32_t* __restrict__ full_num,
+                          int32_t* __restrict__ full_idx, int32_t* __restrict__ bad) {
+    extern __shared__ uint8_t s_code[];   // class of each of the row's UKVB blocks
+    const int i = blockIdx.x, bh = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int s_wp[kThreads / 32], s_wf[kThreads / 32];
+    if (kv_lens) KV_LEN = max(0, min(KV_LEN, kv_lens[bh / maskH]));
+    const int ui = i / rq;
+    const size_t urow = (size_t)bh * UQB + ui;
+    for (int j = tid; j < UKVB; j += kThreads) s_code[j] = kDead;
+    __syncthreads();
+    int n_p = u_kv_num[urow];
+    if (n_p < 0 || n_p > UKVB) {
+        if (tid == 0) atomicExch(bad, 2);
+        n_p = min(max(n_p, 0), UKVB);
+    }
+    for (int n = tid; n < n_p; n += kThreads) {
+        const int j = u_kv_idx[urow * UKVB + n];
+        if (j >= 0 && j < UKVB) s_code[j] = kPartial;
+        else atomicExch(bad, 2);
+    }
+    __syncthreads();
+    if (u_full_num) {
+        int n_f = u_full_num[urow];
+        if (n_f < 0 || n_f > UKVB) {
+            if (tid == 0) atomicExch(bad, 2);
+            n_f = min(max(n_f, 0), UKVB);
+        }
+        for (int n = tid; n < n_f; n += kThreads) {
+            const int j = u_full_idx[urow * UKVB + n];
+            if (j >= 0 && j < UKVB) {
+                if (s_code[j] != kPartial) s_code[j] = kFull;
+            } else {
+                atomicExch(bad, 2);
+            }
+        }
+        __syncthreads();
+    }
+    const size_t row = (size_t)bh * QB + i;
+    int32_t* my_kv = kv_idx + row * KVB;
+    int32_t* my_full = full_idx + row * KVB;
+    const bool q_ragged = (i + 1) * kBlock > Q_LEN;
+    int np = 0, nf = 0;
+    for (int jb = 0; jb < KVB; jb += kThreads) {
+        const int j = jb + tid;
+        int cls = (j < KVB) ? s_code[j / rkv] : kDead;
+        if (j * kBlock >= KV_LEN) cls = kDead;          // past this batch's context
+        if (cls == kFull && (q_ragged || (j + 1) * kBlock > KV_LEN)) cls = kPartial;
+        if (!separate_full && cls == kFull) cls = kPartial;
+        const unsigned bp = __ballot_sync(0xffffffffu, cls == kPartial);
+        const unsigned bf = __ballot_sync(0xffffffffu, cls == kFull);
+        if (lane == 0) {
+            s_wp[warp] = __popc(bp);
+            s_wf[warp] = __popc(bf);
+        }
+        __syncthreads();
+        int op = np, of = nf, tp = 0, tf = 0;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            if (w < warp) {
+                op += s_wp[w];
+                of += s_wf[w];
+            }
+            tp += s_wp[w];
+            tf += s_wf[w];
+        }
+        const unsigned lt = (1u << lane) - 1u;
+        if (cls == kPartial) my_kv[op + __popc(bp & lt)] = j;
+        if (cls == kFull) my_full[of + __popc(bf & lt)] = j;
+        np += tp;
+        nf += tf;
+        __syncthreads();
+    }
+    for (int t = np + tid; t < KVB; t += kThreads) my_kv[t] = 0;
+    for (int t = nf + tid; t < KVB; t += kThreads) my_full[t] = 0;
+    if (tid == 0) {
+        kv_num[row] = np;
+        full_num[row] = nf;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_expand_block_lists(int UQB, int UKVB, int rq, int rkv, int QB, int KVB, int Q_LEN,
+                                      int KV_LEN, const int32_t* kv_lens, int maskH, int maskBH,
+                                      int separate_full,
+                                      const int32_t* u_kv_num, const int32_t* u_kv_idx,
+                                      const int32_t* u_full_num, const int32_t* u_full_idx,
+                                      int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
+                                      int32_t* full_idx, int32_t* bad, cudaStream_t stream) {
+    expand_block_lists_kernel<<<dim3(QB, maskBH), kThreads, UKVB, stream>>>(
+        UQB, UKVB, rq, rkv, QB, KVB, Q_LEN, KV_LEN, kv_lens, maskH, separate_full, u_kv_num, u_kv_idx, u_full_num,
+        u_full_idx, kv_num, kv_idx, full_num, full_idx, bad);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_lists(int QB, int KVB, int maskBH, const int32_t* kv_num,
+                                   const int32_t* kv_idx, const int32_t* full_num,
+                                   const int32_t* full_idx, int32_t* q_num, int32_t* q_idx,
+                                   int32_t* fq_num, int32_t* fq_idx, cudaStream_t stream) {
+    transpose_lists_kernel<<<dim3(KVB, maskBH), kThreads, 0, stream>>>(
+        QB, KVB, kv_num, kv_idx, full_num, full_idx, q_num, q_idx, fq_num, fq_idx, nullptr, nullptr,
+        nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_backward_metadata(int QB, int KVB, int maskBH, int dq_descending,
+                                     const int32_t* kv_num, const int32_t* kv_idx,
+                                     const int32_t* full_num, const int32_t* full_idx,
+                                     const BwdMeta& m, cudaStream_t stream) {
+    // The ranking keeps every unit's cost in shared memory: up to 16384 ints.
+    const int lpt_smem = (QB > KVB ? QB : KVB) * (int)sizeof(int);
+    if (lpt_smem > 48 * 1024) {
+        cudaError_t ea = cudaFuncSetAttribute(lpt_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              lpt_smem);
+        if (ea != cudaSuccess) return ea;
+    }
+    transpose_lists_kernel<<<dim3(KVB, maskBH), kThreads, 0, stream>>>(
+        QB, KVB, kv_num, kv_idx, full_num, full_idx, m.q_num, m.q_idx, m.fq_num, m.fq_idx,
+        m.kv_count, m.kv_cost, m.kv_entries);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    lpt_order_kernel<<<maskBH, 1024, KVB * (int)sizeof(int), stream>>>(KVB, m.kv_cost, m.kv_order);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    dq_entries_kernel<<<dim3(QB, maskBH), kThreads, KVB, stream>>>(
+        QB, KVB, dq_descending, kv_num, kv_idx, full_num, full_idx, m.dq_count, m.dq_cost,
+        m.dq_entries);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    lpt_order_kernel<<<maskBH, 1024, QB * (int)sizeof(int), stream>>>(QB, m.dq_cost, m.dq_order);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_mask_lists(const MaskSpec& spec, int separate_full, int maskBH,
                               int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
                               int32_t* full_idx, int32_t* doc_stats, cudaStream_t stream) {
+    // Per-block document statistics: one array when the query and kv blocks have one size
+    // (max(QB, KVB) entries), else the query blocks' first and the kv blocks' after them.
+    MaskSpec s = spec;
+    s.doc_stats = doc_stats;
+    s.doc_stats_kv = doc_stats;
     if (spec.kind & FA_MASK_DOCUMENT) {
-        const int nblk = spec.QB > spec.KVB ? spec.QB : spec.KVB;
-        doc_block_stats_kernel<<<nblk, kThreads, 0, stream>>>(spec.doc, spec.KV_LEN, nblk,
-                                                              doc_stats);
+        if (spec.BQ == spec.BKV) {
+            const int nblk = spec.QB > spec.KVB ? spec.QB : spec.KVB;
+            doc_block_stats_kernel<<<nblk, kThreads, 0, stream>>>(spec.doc, spec.KV_LEN, nblk, spec.BQ,
+                                                                  doc_stats);
+        } else {
+            s.doc_stats_kv = doc_stats + 3 * (size_t)spec.QB;
+            doc_block_stats_kernel<<<spec.QB, kThreads, 0, stream>>>(spec.doc, spec.KV_LEN, spec.QB,
+                                                                     spec.BQ, doc_stats);
+            cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            doc_block_stats_kernel<<<spec.KVB, kThreads, 0, stream>>>(
+                spec.doc, spec.KV_LEN, spec.KVB, spec.BKV, doc_stats + 3 * (size_t)spec.QB);
+        }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    MaskSpec s = spec;
-    s.doc_stats = doc_stats;
     classify_compact_kernel<<<dim3(spec.QB, maskBH), kThreads, 0, stream>>>(
         s, separate_full, kv_num, kv_idx, full_num, full_idx);
     return cudaGetLastError();
@@ -289,17 +588,20 @@ cudaError_t launch_mask_build(const MaskSpec& spec, int separate_full, int maskB
                               int32_t* full_idx, int32_t* doc_stats, int32_t* sched_count,
                               int32_t* sched_cost, int32_t* sched_entries, int32_t* sched_order,
                               cudaStream_t stream) {
-    if (spec.kind & FA_MASK_DOCUMENT) {
-        const int nblk = spec.QB > spec.KVB ? spec.QB : spec.KVB;
-        doc_block_stats_kernel<<<nblk, kThreads, 0, stream>>>(spec.doc, spec.KV_LEN, nblk,
-                                                              doc_stats);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    classify_compact_kernel<<<dim3(spec.QB, maskBH), kThreads, 0, stream>>>(
-        spec, separate_full, kv_num, kv_idx, full_num, full_idx);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_mask_lists(spec, separate_full, maskBH, kv_num, kv_idx, full_num,
+                                      full_idx, doc_stats, stream);
     if (e != cudaSuccess) return e;
+    e = launch_schedule(spec.QB, spec.KVB, maskBH, NP, kv_num, kv_idx, full_num, full_idx,
+                        sched_count, sched_cost, sched_entries, sched_order, stream);
+    return e;
+}
+
+cudaError_t launch_schedule(int QB, int KVB, int maskBH, int NP, const int32_t* kv_num,
+                            const int32_t* kv_idx, const int32_t* full_num, const int32_t* full_idx,
+                            int32_t* sched_count, int32_t* sched_cost, int32_t* sched_entries,
+                            int32_t* sched_order, cudaStream_t stream) {
+    const MaskSpec spec{0, 0, 0, 0, QB, KVB, kBlock, kBlock, nullptr, nullptr, nullptr, nullptr, 1};
+    cudaError_t e;
     schedule_kernel<<<dim3(NP, maskBH), kThreads, spec.KVB, stream>>>(
         spec.QB, spec.KVB, NP, kv_num, kv_idx, full_num, full_idx, sched_count, sched_cost,
         sched_entries);

@@ -119,8 +119,13 @@ extern "C" fa_status_t fa_create_block_mask_noalloc(
     spec.KV_LEN = KV_LEN;
     spec.QB = QB;
     spec.KVB = KVB;
+    spec.BQ = fa::kBlock;
+    spec.BKV = fa::kBlock;
     spec.doc = (mask_kind & FA_MASK_DOCUMENT) ? params->doc_id : nullptr;
     spec.doc_stats = scratch;
+    spec.doc_stats_kv = scratch;
+    spec.kv_lens = nullptr;
+    spec.maskH = Hm;
     e = fa::launch_mask_lists(spec, sep, Bm * Hm, kv_num_blocks, kv_indices, full_kv_num_blocks,
                               full_kv_indices, scratch, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fa::record_error(FA_ERR_CUDA, cudaGetErrorString(e));

@@ -81,6 +81,13 @@ typedef struct fa_mask_params {
                                              block's dQ over its kv blocks: 1 descending, 0
                                              ascending ("create_block_mask", Parameters,
                                              dq_kv_order; either order is deterministic)          */
+    int32_t        kv_block_size;         /* kv block size of the lists a caller reads back; 0 =
+                                             BLOCK_SIZE ("create_block_mask", Parameters:
+                                             BLOCK_SIZE int or (q, kv) tuple)                     */
+    const int32_t* kv_lens;               /* device, B int32 context lengths, or NULL: key kv of
+                                             batch b exists iff kv < kv_lens[b] (a batch of
+                                             sequences of different lengths, e.g. paged decode);
+                                             needs B > 0.  Copied like doc_id.                   */
 } fa_mask_params_t;
 
 typedef struct fa_score_params {
@@ -113,6 +120,13 @@ typedef struct fa_block_mask_info {
     const int32_t* kv_indices;          /* [B][H][q_blocks][kv_blocks] ascending, zero padded          */
     const int32_t* full_kv_num_blocks;  /* [B][H][q_blocks]            full tiles per query block      */
     const int32_t* full_kv_indices;     /* [B][H][q_blocks][kv_blocks] ascending, zero padded          */
+    /* The same tiles listed per kv block (the transposed lists the backward's dK/dV pass walks): */
+    const int32_t* q_num_blocks;        /* [B][H][kv_blocks]           partial tiles per kv block      */
+    const int32_t* q_indices;           /* [B][H][kv_blocks][q_blocks] ascending, zero padded          */
+    const int32_t* full_q_num_blocks;   /* [B][H][kv_blocks]           full tiles per kv block         */
+    const int32_t* full_q_indices;      /* [B][H][kv_blocks][q_blocks] ascending, zero padded          */
+    int32_t  dq_kv_order;               /* dQ accumulation order over kv blocks: 1 descending, 0 ascending */
+    int32_t  KV_BLOCK_SIZE;             /* kv block size of the lists (BLOCK_SIZE is the query one)   */
 } fa_block_mask_info_t;
 
 /*
@@ -126,9 +140,14 @@ typedef struct fa_block_mask_info {
  *
  *   mask_kind   OR of FA_MASK_* bits (0 = no mask)
  *   params      may be NULL when mask_kind needs neither window nor doc_id
- *               (separate_full_blocks then defaults to 1)
+ *               (separate_full_blocks then defaults to 1, dq_kv_order to 1)
  *   B, H        batch and head extents; 0 means broadcast (stored as 1)
- *   Q_LEN, KV_LEN > 0;  BLOCK_SIZE must be 128 (else FA_ERR_UNSUPPORTED)
+ *   Q_LEN, KV_LEN > 0
+ *   BLOCK_SIZE  query block size of the lists fa_block_mask_get returns; the kv block size is
+ *               params->kv_block_size, or BLOCK_SIZE when that is 0 (the page's int or
+ *               (q, kv) tuple).  Any positive sizes with at most 16384 blocks per side.  The
+ *               kernels always walk their own 128 x 128 tile lists, built alongside, so the
+ *               block size changes what is read back, not the attention result.
  *   out_mask    receives the new mask; release it with fa_destroy_block_mask
  *
  * Work is enqueued on `stream`; the mask may be used by fa_forward on the same stream
@@ -138,6 +157,31 @@ typedef struct fa_block_mask_info {
 fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* params,
                                  int32_t B, int32_t H, int32_t Q_LEN, int32_t KV_LEN,
                                  int32_t BLOCK_SIZE, void* stream, fa_block_mask_t** out_mask);
+
+/*
+ * fa_block_mask_from_kv_blocks -- a block mask from caller-supplied block lists
+ * ("tensorplay.nn.attention.create_block_mask", Parameters, dq_kv_order: explicit schedules
+ * are taken by BlockMask.from_kv_blocks).
+ *
+ *   kv_num_blocks, kv_indices            device int32 [B'][H'][QBu][KVBu] (counts [B'][H'][QBu]):
+ *                                        the partially masked blocks of each query block
+ *   full_kv_num_blocks, full_kv_indices  the same for fully unmasked blocks, or both NULL
+ *                                        (then every listed block is partial)
+ * with B' = max(B, 1), H' = max(H, 1), QBu = ceil(Q_LEN / Q_BLOCK), KVBu = ceil(KV_LEN /
+ * KV_BLOCK).  Q_BLOCK and KV_BLOCK must be multiples of 128 (else FA_ERR_UNSUPPORTED): each
+ * block becomes its 128 x 128 tiles, with the block's class (a ragged tile is never full).
+ * mask_kind and params give the mask_mod applied on partial tiles (0: none, every position
+ * of a listed partial block attends).  Lists need not be sorted; the mask keeps a copy, read
+ * back by fa_block_mask_get.  A count outside [0, KVBu] or an index outside the block grid is
+ * ignored and recorded: fa_get_device_status then returns FA_ERR_INVALID_ARG.
+ */
+fa_status_t fa_block_mask_from_kv_blocks(uint32_t mask_kind, const fa_mask_params_t* params,
+                                         int32_t B, int32_t H, int32_t Q_LEN, int32_t KV_LEN,
+                                         int32_t Q_BLOCK, int32_t KV_BLOCK,
+                                         const int32_t* kv_num_blocks, const int32_t* kv_indices,
+                                         const int32_t* full_kv_num_blocks,
+                                         const int32_t* full_kv_indices, void* stream,
+                                         fa_block_mask_t** out_mask);
 
 /*
  * fa_forward -- fused block-sparse attention forward.
@@ -203,6 +247,60 @@ fa_status_t fa_create_block_mask_noalloc(uint32_t mask_kind, const fa_mask_param
                                          int32_t* full_kv_indices, void* stream);
 
 /*
+ * fa_forward_paged -- fa_forward with the keys and values in pages of a K/V cache: the
+ * PagedAttention pattern expressed through block indices ("PyTorch 2.13 brings custom AI
+ * attention to Mac", "What Attention Patterns Does FlexAttention Support?").
+ *
+ *   k_pages, v_pages   (n_pages, H, 128, D) pools, q's dtype: page p holds 128 consecutive
+ *                      keys of one sequence for every head
+ *   page_table         device int32 [B][page_table_stride]: entry (b, j) is the page holding
+ *                      keys j*128 .. j*128+127 of batch b; page_table_stride >= the mask's
+ *                      kv_blocks; only the entries of listed tiles are read
+ *   block_mask         built for the logical lengths Q_LEN x KV_LEN (usually with kv_lens,
+ *                      one context length per batch element, and no mask kind for decode)
+ * Everything else is fa_forward's.  A page index outside [0, n_pages) reads as zeros and is
+ * recorded: fa_get_device_status then returns FA_ERR_INVALID_ARG.
+ */
+fa_status_t fa_forward_paged(const fa_tensor_t* q, const fa_tensor_t* k_pages,
+                             const fa_tensor_t* v_pages, const int32_t* page_table,
+                             int64_t page_table_stride, const fa_block_mask_t* block_mask,
+                             uint32_t score_mod_kind, const fa_score_params_t* params, float scale,
+                             fa_tensor_t* out, float* lse, void* stream);
+
+/*
+ * fa_backward -- gradients of fa_forward over the same block mask, deterministic.
+ *
+ * Given the forward's out and lse and the upstream gradient dout, writes
+ *   dv = P^T dout,  dq = scale * dS k,  dk = scale * dS^T q,  with
+ *   P = exp(score_mod(scale * q k^T) - lse) on live positions (0 elsewhere),
+ *   dS = P * (dout v^T - rowsum(dout * out)) * score_mod'
+ * ("PyTorch 2.13 brings custom AI attention to Mac", "What Else Shipped in PyTorch 2.13?":
+ * a deterministic FlexAttention backward; "tensorplay.nn.attention.create_block_mask",
+ * Parameters compute_dq_write_order / dq_kv_order: dQ accumulates its kv blocks in a fixed
+ * order).  Here every sum runs in a fixed order on one CTA (no atomics), so repeated calls
+ * give bitwise identical gradients; dQ accumulates in the mask's dq_kv_order.
+ *
+ *   q, k, v, out, lse, block_mask, score_mod_kind, params, scale: as passed to fa_forward,
+ *               with out and lse the forward's results (lse must not be NULL here)
+ *   dout        (B, H, Q_LEN, D), q's dtype
+ *   dq          (B, H, Q_LEN, D); dk, dv (B, H, KV_LEN, D); q's dtype, caller-owned
+ *   workspace   device scratch of at least fa_backward_workspace_bytes(B, H, Q_LEN) bytes,
+ *               16-byte aligned, caller-owned; the call leaves nothing in it that a later call
+ *               needs.  Calls that overlap on the GPU need distinct workspaces.
+ *
+ * Three kernels run on `stream`: a pre-pass (rowsum(dout * out) and lse into the workspace),
+ * the dK/dV pass (one unit per kv block) and the dQ pass (one unit per query block).  Shapes,
+ * dtypes and limits are fa_forward's.  Device-side waits are bounded as in fa_forward.
+ */
+size_t fa_backward_workspace_bytes(int64_t B, int64_t H, int64_t Q_LEN);
+fa_status_t fa_backward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tensor_t* v,
+                        const fa_tensor_t* out, const fa_tensor_t* dout, const float* lse,
+                        const fa_block_mask_t* block_mask, uint32_t score_mod_kind,
+                        const fa_score_params_t* params, float scale, fa_tensor_t* dq,
+                        fa_tensor_t* dk, fa_tensor_t* dv, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
  * fa_masked_softmax -- the causal-masked softmax over materialised scores, in one kernel.
  *
  * probs[b,h,q,kv] = softmax over kv of  (q + offset >= kv ? scores[b,h,q,kv] : finfo.min)
@@ -240,8 +338,10 @@ fa_status_t fa_block_mask_get(const fa_block_mask_t* block_mask, fa_block_mask_i
 
 /*
  * Synchronise `stream`, read and clear the device status word that kernels using this
- * mask write when a bounded device-side wait runs out.  Returns FA_OK, FA_ERR_TIMEOUT,
- * or FA_ERR_CUDA if the stream itself reports an error.
+ * mask write when a bounded device-side wait runs out, or that fa_block_mask_from_kv_blocks
+ * writes when the caller's lists were out of range, or fa_forward_paged when a page index
+ * was.  Returns FA_OK, FA_ERR_TIMEOUT, FA_ERR_INVALID_ARG (lists or pages out of range), or
+ * FA_ERR_CUDA if the stream reports an error.
  */
 fa_status_t fa_get_device_status(const fa_block_mask_t* block_mask, void* stream);
 

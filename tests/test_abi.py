@@ -66,8 +66,10 @@ def _create(fa, kind, params, B=0, H=0, Q=256, KV=256, BS=128):
 def test_create_block_mask_rejects_bad_arguments(fa):
     P = fa.FaMaskParams
     assert fa._lib.fa_create_block_mask(1, None, 0, 0, 256, 256, 128, None, None) == fa.FA_ERR_INVALID_ARG
-    assert _create(fa, 1, None, BS=64)[0] == fa.FA_ERR_UNSUPPORTED
-    assert "BLOCK_SIZE" in fa.fa_last_error_message()
+    assert _create(fa, 1, None, BS=0)[0] == fa.FA_ERR_INVALID_ARG      # block sizes are positive
+    assert "block sizes" in fa.fa_last_error_message()
+    assert _create(fa, 1, None, BS=1, Q=16385, KV=16385)[0] == fa.FA_ERR_UNSUPPORTED
+    assert "blocks per side" in fa.fa_last_error_message()
     assert _create(fa, 8, None)[0] == fa.FA_ERR_INVALID_ARG          # unknown kind bit
     assert _create(fa, 2, P(0, None, 1))[0] == fa.FA_ERR_INVALID_ARG  # window must be > 0
     assert _create(fa, 2, None)[0] == fa.FA_ERR_INVALID_ARG          # window missing
@@ -124,8 +126,14 @@ def test_null_handles_are_rejected_or_ignored(fa):
 
 def test_python_binding_raises_fa_error(fa):
     with pytest.raises(fa.FaError) as ei:
-        fa.fa_create_block_mask(1, None, 0, 0, 256, 256, BLOCK_SIZE=64, stream=0)
-    assert ei.value.status == fa.FA_ERR_UNSUPPORTED
+        fa.fa_create_block_mask(1, None, 0, 0, 256, 256, BLOCK_SIZE=0, stream=0)
+    assert ei.value.status == fa.FA_ERR_INVALID_ARG
+    # Caller block lists must come in multiples of the kernels' 128 x 128 tiles.
+    dummy = ctypes.c_void_p(0x1000)
+    h = ctypes.c_void_p()
+    st = fa._lib.fa_block_mask_from_kv_blocks(1, None, 0, 0, 256, 256, 64, 128, dummy, dummy, None,
+                                              None, None, ctypes.byref(h))
+    assert st == fa.FA_ERR_UNSUPPORTED
 
 
 def _header_constants():
@@ -149,12 +157,12 @@ def test_binding_constants_match_the_header(fa):
 
 def test_struct_layouts_match_the_header(fa):
     # ctypes mirrors of the ABI structs: field order and sizes as declared (64-bit ABI).
-    assert ctypes.sizeof(fa.FaMaskParams) == 24      # int32, pad, void*, int32, int32
+    assert ctypes.sizeof(fa.FaMaskParams) == 40      # int32, pad, void*, int32 x 3, pad, void*
     assert ctypes.sizeof(fa.FaScoreParams) == 16     # float, pad, const float*
     assert ctypes.sizeof(fa.FaTensor) == 8 + 8 + 4 * 8 + 4 * 8
     text = open(os.path.join(ROOT, "include", "fa_b200.h")).read()
     for struct, fields in (("fa_mask_params", ["window", "doc_id", "separate_full_blocks",
-                                               "dq_kv_order"]),
+                                               "dq_kv_order", "kv_block_size", "kv_lens"]),
                            ("fa_score_params", ["softcap", "alibi_slopes"]),
                            ("fa_tensor", ["data", "dtype", "B", "stride"])):
         body = re.search(r"typedef struct %s \{(.*?)\}" % struct, text, flags=re.S).group(1)

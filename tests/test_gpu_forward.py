@@ -358,3 +358,50 @@ def test_host_buffers_are_rejected_before_any_launch():
     w = wl.Workload("host_check", B=1, H=2, S=256, D=64, dtype="bf16", mask_kind=C, seed=26)
     O, L = run_oracle(w, q, k, v)
     compare(out, lse, O, L)
+
+
+def test_per_batch_sequence_lengths():
+    # kv_lens: key kv of batch b exists iff kv < kv_lens[b]; the mask is per batch element.
+    fa = fa_module()
+    lens = np.array([300, 1000, 129], dtype=np.int32)
+    w = wl.Workload("lens", B=3, H=2, S=1000, D=128, dtype="bf16", mask_kind=C, seed=29)
+    q, k, v = wl.make_qkv(w)
+    bm = fa.create_block_mask(C, 3, None, 1000, 1000, kv_lens=torch.from_numpy(lens).cuda())
+    ref = oracle.create_block_mask(oracle.make_mask_mod(C, kv_lens=lens), 3, None, 1000, 1000)
+    from gpu_common import assert_block_mask_equal
+    assert_block_mask_equal(bm, ref)
+    out, lse = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm)
+    torch.cuda.synchronize()
+    mm = oracle.make_mask_mod(C, kv_lens=lens)
+    O, L = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), mm, None, scale=w.scale)
+    compare(out, lse, O, L)
+
+
+@pytest.mark.parametrize("Q", [1, 5])
+def test_paged_decode_equals_contiguous_and_the_oracle(Q):
+    # PagedAttention through block indices: K/V in shuffled 128-token pages of one pool.
+    fa = fa_module()
+    dw = wl.DecodeWorkload("decode_small", B=4, H=4, D=128, lo=130, hi=2500, Q=Q, seed=30)
+    q, k, v, kp, vp, table, lens = wl.make_decode(dw)
+    KV = k.shape[2]
+    lens_t = torch.from_numpy(lens).cuda()
+    bm = fa.create_block_mask(0, dw.B, None, Q, KV, kv_lens=lens_t)
+    paged = fa.flex_attention(q.cuda(), kp.cuda(), vp.cuda(), bm, page_table=table.cuda())
+    contig = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm)
+    torch.cuda.synchronize()
+    assert bm.device_status() == fa.FA_OK
+    assert torch.equal(paged[0], contig[0]) and torch.equal(paged[1], contig[1])
+    mm = oracle.make_mask_mod(0, kv_lens=lens)
+    O, L = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), mm, None, scale=dw.scale)
+    compare(paged[0], paged[1], O, L)
+
+
+def test_paged_page_out_of_range_is_reported():
+    fa = fa_module()
+    dw = wl.DecodeWorkload("decode_bad", B=2, H=2, D=64, lo=200, hi=300, seed=31)
+    q, k, v, kp, vp, table, lens = wl.make_decode(dw)
+    table[1, 0] = kp.shape[0] + 5
+    bm = fa.create_block_mask(0, dw.B, None, 1, k.shape[2], kv_lens=torch.from_numpy(lens).cuda())
+    fa.flex_attention(q.cuda(), kp.cuda(), vp.cuda(), bm, page_table=table.cuda())
+    assert bm.device_status() == fa.FA_ERR_INVALID_ARG
+    assert bm.device_status() == fa.FA_OK

@@ -19,6 +19,13 @@ Recipe (the same for every workload):
     bf16.  Q is a chunk of 1024 query rows that closes a context of K keys, so the causal
     offset is K - Q (the 8K and 32K sequences of "Fuse the causal mask into the SDPA
     fallback softmax", MLX pull request 3919).
+  * The decode workloads hold a batch of B sequences with seeded context lengths
+    (``numpy.random.default_rng(seed).integers(lo, hi + 1, B)``), one new query token per
+    sequence, and the keys and values in 128-token pages of one shared pool, placed by a
+    seeded random permutation of the pages (PagedAttention through block indices, "PyTorch
+    2.13 brings custom AI attention to Mac", "What Attention Patterns Does FlexAttention
+    Support?").  q, k, v are drawn like the other workloads' (q of shape (B, H, 1, D), k and v
+    of shape (B, H, max length, D)); the pool takes each sequence's pages from k and v.
   * The document-packed workload splits T = 8192 positions into 4 documents of
     seeded random lengths, each at least 512 long: three cut points drawn from
     ``numpy.random.default_rng(seed).integers(0, 6145, 3)`` and sorted give the
@@ -190,3 +197,66 @@ def make_scores(w: SoftmaxWorkload, seed: Optional[int] = None):
     g.manual_seed(w.seed if seed is None else seed)
     t = torch.randn((w.B, w.H, w.Q, w.K), generator=g, dtype=torch.float32)
     return t.to(torch_dtype(w.dtype))
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    """One decode step: B sequences of seeded lengths in [lo, hi], paged K/V, Q_LEN new tokens."""
+    name: str
+    B: int
+    H: int
+    D: int
+    lo: int
+    hi: int
+    Q: int = 1
+    dtype: str = "bf16"
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.D))
+
+    def lengths(self) -> np.ndarray:
+        return np.random.default_rng(self.seed).integers(self.lo, self.hi + 1, self.B).astype(np.int32)
+
+    @property
+    def kv_len(self) -> int:
+        return int(self.lengths().max())
+
+
+DECODE_WORKLOADS = [
+    DecodeWorkload("decode_paged_b16h16_d128_ctx1k-8k_bf16", B=16, H=16, D=128, lo=1024, hi=8192,
+                   seed=71),
+]
+
+
+def make_decode(w: DecodeWorkload):
+    """q (B, H, Q, D), contiguous k, v (B, H, KV, D), page pools (n_pages, H, 128, D) and the page
+    table (B, ceil(KV / 128)) int32, plus the lengths; all on the CPU."""
+    import torch
+    lens = w.lengths()
+    KV = int(lens.max())
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    td = torch_dtype(w.dtype)
+    q = torch.randn((w.B, w.H, w.Q, w.D), generator=g, dtype=torch.float32).to(td)
+    k = torch.randn((w.B, w.H, KV, w.D), generator=g, dtype=torch.float32).to(td)
+    v = torch.randn((w.B, w.H, KV, w.D), generator=g, dtype=torch.float32).to(td)
+    nblk = -(-KV // 128)
+    pages_per = [-(-int(n) // 128) for n in lens]
+    n_pages = sum(pages_per)
+    perm = np.random.default_rng(w.seed + 1).permutation(n_pages).astype(np.int32)
+    table = np.zeros((w.B, nblk), dtype=np.int32)
+    kp = torch.zeros((n_pages, w.H, 128, w.D), dtype=td)
+    vp = torch.zeros((n_pages, w.H, 128, w.D), dtype=td)
+    nxt = 0
+    for b in range(w.B):
+        for j in range(pages_per[b]):
+            page = int(perm[nxt])
+            nxt += 1
+            table[b, j] = page
+            rows = slice(j * 128, min((j + 1) * 128, KV))
+            n = rows.stop - rows.start
+            kp[page, :, :n] = k[b, :, rows]
+            vp[page, :, :n] = v[b, :, rows]
+    return q, k, v, kp, vp, torch.from_numpy(table), lens
