@@ -15,7 +15,10 @@ import ctypes
 import os
 from typing import Optional, Tuple
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libfa_b200.so")
+# FA_B200_LIBRARY may name another build of the same library (build.py --debug writes
+# _lib/libfa_b200_debug.so, whose kernels check metadata indices); the default is the product.
+_LIB_PATH = os.environ.get("FA_B200_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "_lib", "libfa_b200.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
         f"{_LIB_PATH} is missing: build it with `python block_sparse_masked_x128_b200/build.py`")

@@ -1,6 +1,6 @@
 """Build the sm_100a shared library in-tree: block_sparse_masked_x128_b200/_lib/libfa_b200.so.
 
-    python block_sparse_masked_x128_b200/build.py [--verbose] [--ptxas-info] [--force]
+    python block_sparse_masked_x128_b200/build.py [--verbose] [--ptxas-info] [--force] [--debug]
 
 (Run it as a file, not as a package module: importing the package loads the library.)
 
@@ -27,6 +27,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libfa_b200.so")
 TRACE_LIB = os.path.join(LIBDIR, "libfa_b200_trace.so")
+DEBUG_LIB = os.path.join(LIBDIR, "libfa_b200_debug.so")
 SOURCES = ["api.cu", "mask_builder.cu", "attn_fwd.cu", "noalloc.cu", "masked_softmax.cu", "attn_bwd.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -38,13 +39,15 @@ def _nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _flags(ptxas_info: bool, trace: bool = False) -> list:
+def _flags(ptxas_info: bool, trace: bool = False, debug: bool = False) -> list:
     f = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
                 "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]
     if ptxas_info:
         f += ["-Xptxas", "-v"]
     if trace:
         f += ["-DFA_TRACE"]
+    if debug:
+        f += ["-DFA_DEBUG"]
     return f
 
 
@@ -67,13 +70,15 @@ def _compile(src: str, flags: list, force: bool, build_dir: str = BUILD) -> tupl
 
 
 def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False,
-          trace: bool = False) -> str:
-    """Build the library; with trace=True build the phase-tracing variant instead."""
-    build_dir = os.path.join(BUILD, "trace") if trace else BUILD
-    lib = TRACE_LIB if trace else LIB
+          trace: bool = False, debug: bool = False) -> str:
+    """Build the library; trace=True builds the phase-tracing variant, debug=True the variant
+    whose kernels check metadata indices (FA_DEBUG), each under its own name."""
+    variant = "trace" if trace else ("debug" if debug else "")
+    build_dir = os.path.join(BUILD, variant) if variant else BUILD
+    lib = TRACE_LIB if trace else (DEBUG_LIB if debug else LIB)
     os.makedirs(build_dir, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
-    flags = _flags(ptxas_info, trace)
+    flags = _flags(ptxas_info, trace, debug)
     with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
         results = list(ex.map(lambda s: _compile(s, flags, force or ptxas_info, build_dir), SOURCES))
     objs = [o for o, _ in results]
@@ -96,8 +101,10 @@ def main(argv=None) -> int:
     ap.add_argument("--ptxas-info", action="store_true")
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--trace", action="store_true", help="build the phase-tracing variant")
+    ap.add_argument("--debug", action="store_true",
+                    help="build the variant whose kernels check metadata indices (FA_DEBUG)")
     a = ap.parse_args(argv)
-    print(build(a.verbose, a.ptxas_info, a.force, a.trace))
+    print(build(a.verbose, a.ptxas_info, a.force, a.trace, a.debug))
     return 0
 
 

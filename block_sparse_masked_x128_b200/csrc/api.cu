@@ -8,9 +8,18 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "fa_internal.h"
 
 namespace {
+
+// An NVTX range over a host entry point (what a profiler's timeline shows as the call that
+// enqueued the kernels); costs a few nanoseconds when no tool listens.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
 
 thread_local std::string g_last_error;
 std::atomic<int> g_stall_loads{0};
@@ -392,6 +401,7 @@ extern "C" {
 fa_status_t fa_create_block_mask(uint32_t mask_kind, const fa_mask_params_t* params, int32_t B,
                                  int32_t H, int32_t Q_LEN, int32_t KV_LEN, int32_t BLOCK_SIZE,
                                  void* stream, fa_block_mask_t** out_mask) {
+    NvtxRange nvtx_range("fa_create_block_mask");
     if (!out_mask) return fail(FA_ERR_INVALID_ARG, "out_mask is NULL");
     *out_mask = nullptr;
     fa_status_t s = check_mask_args(mask_kind, params, B, H, Q_LEN, KV_LEN);
@@ -436,6 +446,7 @@ fa_status_t fa_block_mask_from_kv_blocks(uint32_t mask_kind, const fa_mask_param
                                          const int32_t* kv_indices, const int32_t* full_kv_num_blocks,
                                          const int32_t* full_kv_indices, void* stream,
                                          fa_block_mask_t** out_mask) {
+    NvtxRange nvtx_range("fa_block_mask_from_kv_blocks");
     if (!out_mask) return fail(FA_ERR_INVALID_ARG, "out_mask is NULL");
     *out_mask = nullptr;
     fa_status_t s = check_mask_args(mask_kind, params, B, H, Q_LEN, KV_LEN);
@@ -540,6 +551,8 @@ fa_status_t fa_get_device_status(const fa_block_mask_t* m, void* stream) {
         if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
         if (h == 2)
             return fail(FA_ERR_INVALID_ARG, "the caller's block lists held a count or index outside the block grid");
+        if (h == fa::kStatusBadIndex)
+            return fail(FA_ERR_INTERNAL, "a kernel met a metadata index out of range (debug build check)");
         return fail(FA_ERR_TIMEOUT, "a device-side wait ran past its limit (status %d)", h);
     }
     return ok();
@@ -683,6 +696,7 @@ fa_status_t fa_backward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_ten
                         const fa_score_params_t* params, float scale, fa_tensor_t* dq,
                         fa_tensor_t* dk, fa_tensor_t* dv, void* workspace, size_t workspace_bytes,
                         void* stream) {
+    NvtxRange nvtx_range("fa_backward");
     fa_status_t s;
     const fa_tensor_t* all[8] = {q, k, v, out, dout, dq, dk, dv};
     const char* names[8] = {"q", "k", "v", "out", "dout", "dq", "dk", "dv"};
@@ -817,6 +831,7 @@ fa_status_t fa_backward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_ten
 
 fa_status_t fa_masked_softmax(const fa_tensor_t* scores, uint32_t mask_kind, int64_t offset,
                               fa_tensor_t* probs, void* stream) {
+    NvtxRange nvtx_range("fa_masked_softmax");
     fa_status_t s;
     if ((s = check_tensor(scores, "scores")) != FA_OK) return s;
     if ((s = check_tensor(probs, "probs")) != FA_OK) return s;
@@ -869,6 +884,7 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
                        const fa_block_mask_t* m, uint32_t score_mod_kind,
                        const fa_score_params_t* params, float scale, fa_tensor_t* out, float* lse,
                        void* stream) {
+    NvtxRange nvtx_range("fa_forward");
     return forward_impl(q, k, v, nullptr, 0, m, score_mod_kind, params, scale, out, lse, stream);
 }
 
@@ -877,6 +893,7 @@ fa_status_t fa_forward_paged(const fa_tensor_t* q, const fa_tensor_t* k_pages,
                              int64_t page_table_stride, const fa_block_mask_t* m,
                              uint32_t score_mod_kind, const fa_score_params_t* params, float scale,
                              fa_tensor_t* out, float* lse, void* stream) {
+    NvtxRange nvtx_range("fa_forward_paged");
     if (!page_table) return fail(FA_ERR_INVALID_ARG, "page_table is NULL");
     if ((reinterpret_cast<uintptr_t>(page_table) & 3u) != 0)
         return fail(FA_ERR_INVALID_ARG, "page_table is not 4-byte aligned");

@@ -109,7 +109,9 @@ __device__ __forceinline__ BUnit decode_bunit(const BwdParams& p, int u) {
     const int mb = (p.maskB == 1) ? 0 : un.b, mh = (p.maskH == 1) ? 0 : un.h;
     const size_t base = ((size_t)mb * p.maskH + mh) * p.units_per_bh;
     un.idx = __ldg(p.order + base + r);
+    FA_DCHECK_INDEX(un.idx, p.units_per_bh, p.status);
     un.E = __ldg(p.count + base + un.idx);
+    FA_DCHECK_INDEX(un.E, p.entries_stride + 1, p.status);
     un.entries = p.entries + (base + un.idx) * (size_t)p.entries_stride;
     return un;
 }
@@ -197,7 +199,8 @@ __device__ void bwd_producer(const BwdParams& p, const CUtensorMap* tq, const CU
         er.init(un.entries, un.E);
         const size_t vec_row = ((size_t)un.b * p.H + un.h) * (size_t)p.q_pad;
         for (int e = 0; e < un.E; ++e) {
-            const int t = er.get(e) & 0xFFFF;
+            int t = er.get(e) & 0xFFFF;
+            FA_DCHECK_INDEX(t, p.entries_stride, p.status);
             const int s = (int)(pos % C::kStages);
             if (!wait(C::kBarSlotEmpty + s, ((pos / C::kStages) & 1u) ^ 1u)) { ok = false; break; }
             const uint32_t dst = sbase + C::kStageOff + (uint32_t)s * C::kStageBytes;
@@ -402,7 +405,8 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
         er.init(un.entries, un.E);
         for (int e = 0; e < un.E; ++e) {
             const int code = er.get(e);
-            const int t = code & 0xFFFF;
+            int t = code & 0xFFFF;
+            FA_DCHECK_INDEX(t, p.entries_stride, p.status);
             const bool full = (code & kFull0) != 0;
             const int s = (int)(pos % C::kStages);
             ++pos;

@@ -287,9 +287,17 @@ __device__ __forceinline__ float2 softmax_p_row(const float2 (&x)[64], float2 nb
     return __fadd2_rn(__fadd2_rn(rs[0], rs[1]), __fadd2_rn(rs[2], rs[3]));
 }
 
-// VAR = score_mod bits (FA_SCORE_*) | kVarDocument when the mask has a document predicate:
-// both are compile-time, so kernels without them carry none of their registers.
+// VAR = score_mod bits (FA_SCORE_*) | kVarDocument when the mask has a document predicate
+// | kVarFixedMax for the fixed-max soft-cap variant: all compile-time, so kernels without them
+// carry none of their registers.
 constexpr int kVarDocument = 4;
+// Fixed max (bf16 with a soft-cap, every live score <= cap): P = 2^(x - cap log2 e) <= 1 with no
+// row max and no rescale.  Without ALiBi every live score is >= -cap; with it the bias must not
+// be positive (causal-type masks, the default positive slopes) and each query row keeps its
+// own key, whose bias is 0.  Either way a row's sum is >= e^(-2 cap), a normal float32 and
+// bfloat16 value for caps up to 32 (e^-60 at cap 30), and a key the fixed base drives below
+// the float range weighs less than 2^-39 of that row's largest term.
+constexpr int kVarFixedMax = 8;
 
 template <int D, bool BF16, int VAR>
 __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t tmem,
@@ -297,6 +305,8 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
     using C = Cfg<D>;
     constexpr int SCORE = VAR & (FA_SCORE_SOFTCAP | FA_SCORE_ALIBI);
     constexpr bool kDoc = (VAR & kVarDocument) != 0;
+    constexpr bool kFixedMax = (VAR & kVarFixedMax) != 0;
+    static_assert(!kFixedMax || (SCORE & FA_SCORE_SOFTCAP), "fixed max needs the soft-cap bound");
     const int wq = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant this warp may access
     const int lane = threadIdx.x & 31;
     const int row = wq * 32 + lane;
@@ -355,7 +365,8 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
         for (int e = 0; e < un.E; ++e) {
             const int code = er.get(e);
             if (!(code & live_bit)) continue;
-            const int j = code & 0xFFFF;
+            int j = code & 0xFFFF;
+            FA_DCHECK_INDEX(j, p.KVB, p.status);
             const bool full = (code & full_bit) != 0;
             FA_TRACE_EV(tslot, 1);
             if (!wait(kBarSFull + t, sf_cnt & 1u)) { ok = false; break; }
@@ -434,26 +445,31 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                     }
                 }
             }
-            // Row max with three-input max: eight independent chains over eighths.
-            float mc[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) mc[c] = fmaxf(x[8 * c].x, x[8 * c].y);
-#pragma unroll
-            for (int i = 1; i < 8; ++i)
-#pragma unroll
-                for (int c = 0; c < 8; ++c) mc[c] = max3(mc[c], x[8 * c + i].x, x[8 * c + i].y);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) mc[c] = fmaxf(mc[c], mc[c + 4]);
-            float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
-            if constexpr (SCORE == 0) mt *= p.scale_log2;
-            const float m_new = fmaxf(m, mt);
-            FA_TRACE_EV(tslot, 4);
-            const bool need = m_new > m + kRescaleThreshold;
-            const bool any_need = __any_sync(kFullMask, need);
+            bool any_need = false;
             float alpha = 1.0f;
-            if (need) {
-                alpha = ex2_approx(m - m_new);  // m = -inf gives 0 (l and O are empty then)
-                m = m_new;
+            if constexpr (kFixedMax) {
+                m = p.softcap_log2;          // the bound of every live score
+            } else {
+                // Row max with three-input max: eight independent chains over eighths.
+                float mc[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) mc[c] = fmaxf(x[8 * c].x, x[8 * c].y);
+#pragma unroll
+                for (int i = 1; i < 8; ++i)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) mc[c] = max3(mc[c], x[8 * c + i].x, x[8 * c + i].y);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) mc[c] = fmaxf(mc[c], mc[c + 4]);
+                float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+                if constexpr (SCORE == 0) mt *= p.scale_log2;
+                const float m_new = fmaxf(m, mt);
+                FA_TRACE_EV(tslot, 4);
+                const bool need = m_new > m + kRescaleThreshold;
+                any_need = __any_sync(kFullMask, need);
+                if (need) {
+                    alpha = ex2_approx(m - m_new);  // m = -inf gives 0 (l and O are empty then)
+                    m = m_new;
+                }
             }
             const float base = (m == -INFINITY) ? 0.f : m;
             FA_TRACE_EV(tslot, 9);
@@ -622,16 +638,30 @@ cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMa
 cudaError_t launch_attn_fwd(const FwdParams& p, int D, bool bf16, int score_kind,
                             const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             int grid, cudaStream_t stream) {
-    const int var = score_kind | ((p.mask_kind & FA_MASK_DOCUMENT) ? kVarDocument : 0);
+    int var = score_kind | ((p.mask_kind & FA_MASK_DOCUMENT) ? kVarDocument : 0);
+    // The fixed-max variant: bf16 (P keeps float32's exponent range) and a soft-cap of at most
+    // 32 (so e^(-2 cap) stays a normal float), and with ALiBi a bias that cannot be positive
+    // (a causal-type mask, the default positive slopes) and every query row's own key, whose
+    // bias is 0, inside the context (no per-batch lengths, Q_LEN <= KV_LEN).  Without ALiBi
+    // every live score is >= -cap, so any row with a live key keeps its sum that large.
+    const bool causal_type = (p.mask_kind & (FA_MASK_CAUSAL | FA_MASK_SLIDING_WINDOW)) != 0;
+    if (bf16 && (score_kind & FA_SCORE_SOFTCAP) && p.softcap <= 32.0f &&
+        (!(score_kind & FA_SCORE_ALIBI) ||
+         (causal_type && !p.alibi_slopes && !p.kv_lens && p.Q_LEN <= p.KV_LEN)))
+        var |= kVarFixedMax;
 #define FA_CASE(DD, BB, VV)                                                 \
     if (D == DD && bf16 == BB && var == VV)                                 \
         return launch_t<DD, BB, VV>(p, tq, tk, tv, grid, stream);
 #define FA_CASES(DD, BB) FA_CASE(DD, BB, 0) FA_CASE(DD, BB, 1) FA_CASE(DD, BB, 2) FA_CASE(DD, BB, 3) \
     FA_CASE(DD, BB, 4) FA_CASE(DD, BB, 5) FA_CASE(DD, BB, 6) FA_CASE(DD, BB, 7)
+#define FA_FIXED(DD) FA_CASE(DD, true, 9) FA_CASE(DD, true, 11) FA_CASE(DD, true, 13) FA_CASE(DD, true, 15)
     FA_CASES(64, true)
     FA_CASES(64, false)
     FA_CASES(128, true)
     FA_CASES(128, false)
+    FA_FIXED(64)
+    FA_FIXED(128)
+#undef FA_FIXED
 #undef FA_CASES
 #undef FA_CASE
     return cudaErrorInvalidValue;

@@ -17,6 +17,25 @@ namespace fa {
 constexpr int kBlock = 128;          // BLOCK_SIZE: query rows and keys per tile
 constexpr int kMaxBlocks = 16384;    // q_blocks and kv_blocks limit (2M positions)
 
+// Debug builds (FA_DEBUG, build.py --debug): kernels check each index they read from the
+// mask's metadata before using it; an index out of range is recorded in the mask's status
+// word (kStatusBadIndex) and replaced by 0, so the kernel finishes instead of faulting.  The
+// product build compiles the checks away.
+constexpr int kStatusBadIndex = 3;
+#ifdef FA_DEBUG
+#define FA_DCHECK_INDEX(idx, limit, status)                              \
+    do {                                                                 \
+        if ((unsigned)(idx) >= (unsigned)(limit)) {                      \
+            atomicExch((status), kStatusBadIndex);                       \
+            (idx) = 0;                                                   \
+        }                                                                \
+    } while (0)
+#else
+#define FA_DCHECK_INDEX(idx, limit, status) \
+    do {                                    \
+    } while (0)
+#endif
+
 // Tile classes written by the mask builder.
 constexpr int kDead = 0, kPartial = 1, kFull = 2, kAmbiguous = 3;
 

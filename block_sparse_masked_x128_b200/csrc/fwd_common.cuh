@@ -53,8 +53,10 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     un.b = b;
     un.h = h;
     un.pair = __ldg(p.sched_order + sidx * p.NP + r);
+    FA_DCHECK_INDEX(un.pair, p.NP, p.status);
     const int2 c = __ldg(reinterpret_cast<const int2*>(p.sched_count) + sidx * p.NP + un.pair);
     un.E = c.x;
+    FA_DCHECK_INDEX(un.E, p.KVB + 1, p.status);
     un.nl0 = c.y & 0xFFFF;
     un.nl1 = (int)((unsigned)c.y >> 16);
     un.entries = p.sched_entries + (sidx * p.NP + un.pair) * (size_t)p.KVB;
@@ -191,7 +193,8 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
         EntryReader er;
         er.init(un.entries, un.E);
         for (int e = 0; e < un.E && ok; ++e) {
-            const int j = er.get(e) & 0xFFFF;
+            int j = er.get(e) & 0xFFFF;
+            FA_DCHECK_INDEX(j, p.KVB, p.status);
             // K_j and V_j: rows j*128.. of batch b, or with paged K/V the page the table gives
             // for (b, j) (a page outside the pools is recorded and reads as zeros).
             int kv_row = j * kBlock, kv_batch = un.b;
