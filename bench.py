@@ -728,7 +728,10 @@ def main(argv=None) -> int:
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true",
-                    help="time only --workload (skip the per_workload section)")
+                    help="time only --workload (skip the per_workload and next_rows sections)")
+    ap.add_argument("--only", choices=["masked_softmax", "decode", "backward"],
+                    help="time only this row and print its line (for profiling one kernel); "
+                         "backward runs on --workload")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-budget-s", type=float, default=60.0)
     args = ap.parse_args(argv)
@@ -753,7 +756,20 @@ def main(argv=None) -> int:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     try:
-        res = run_ours(args, w, world, rank, local)
+        if args.only:
+            import torch
+            torch.cuda.set_device(local)
+            dev = torch.device("cuda", local)
+            if args.only == "masked_softmax":
+                res = time_masked_softmax(wl.SOFTMAX_WORKLOADS[0], args.steps, args.warmup, world, dev)
+            elif args.only == "decode":
+                res = time_decode(wl.DECODE_WORKLOADS[0], args.steps, args.warmup, world, dev)
+            else:
+                res = time_backward(w, args.steps, args.warmup, world, rank, dev)
+            res.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                        "higher_is_better": True, "scaling": "weak", "data": "synthetic"})
+        else:
+            res = run_ours(args, w, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist
