@@ -265,6 +265,8 @@ fa_status_t allocate_mask(uint32_t mask_kind, const fa_mask_params_t* params, in
     const size_t o_udst = take((has_doc && user) ? (size_t)(UQB + UKVB) * 3 * 4 : 0);
     const size_t o_sc = take(BH * NP * 8), o_scost = take(BH * NP * 4);
     const size_t o_se = take(BH * NP * KVB * 4), o_so = take(BH * NP * 4);
+    const bool global_order = BH * NP <= (size_t)fa::kGlobalOrderMax;
+    const size_t o_sgo = take(global_order ? BH * NP * 4 : 0);
     const size_t n_kv = BH * KVB, n_q = BH * QB, n_tiles = BH * QB * KVB;
     const size_t o_qn = take(n_kv * 4), o_qi = take(n_tiles * 4), o_fqn = take(n_kv * 4),
                  o_fqi = take(n_tiles * 4);
@@ -313,6 +315,7 @@ fa_status_t allocate_mask(uint32_t mask_kind, const fa_mask_params_t* params, in
     m->sched_cost = at(o_scost);
     m->sched_entries = at(o_se);
     m->sched_order = at(o_so);
+    m->sched_gorder = global_order ? at(o_sgo) : nullptr;
     m->dq_kv_order = params ? (params->dq_kv_order ? 1 : 0) : 1;
     m->bwd = fa::BwdMeta{at(o_qn),  at(o_qi),     at(o_fqn), at(o_fqi), at(o_kvc),    at(o_kvcost),
                          at(o_kve), at(o_kvo),    at(o_dqc), at(o_dqcost), at(o_dqe), at(o_dqo)};
@@ -371,6 +374,8 @@ cudaError_t build_derived(fa_block_mask_t* m, cudaStream_t st) {
     cudaError_t e = fa::launch_schedule(m->QB, m->KVB, BH, m->NP, m->kv_num, m->kv_idx, m->full_num,
                                         m->full_idx, m->sched_count, m->sched_cost, m->sched_entries,
                                         m->sched_order, st);
+    if (e != cudaSuccess) return e;
+    if (m->sched_gorder) e = fa::launch_global_order(BH * m->NP, m->sched_cost, m->sched_gorder, st);
     if (e != cudaSuccess) return e;
     return fa::launch_backward_metadata(m->QB, m->KVB, BH, m->dq_kv_order, m->kv_num, m->kv_idx,
                                         m->full_num, m->full_idx, m->bwd, st);
@@ -652,6 +657,7 @@ fa_status_t forward_impl(const fa_tensor_t* q, const fa_tensor_t* k, const fa_te
     p.page_stride = (int32_t)(page_table ? page_stride : 0);
     p.n_pages = (int32_t)(page_table ? k->B : 0);
     p.sched_order = m->sched_order;
+    p.sched_gorder = m->sched_gorder;
     p.sched_count = m->sched_count;
     p.sched_entries = m->sched_entries;
     p.scale = sc;

@@ -73,6 +73,7 @@ struct FwdParams {
     int32_t page_stride;
     int32_t n_pages;              // pages in the K/V pools (the pools' batch extent)
     const int32_t* sched_order;   // [maskB*maskH][NP]  pairs by descending cost
+    const int32_t* sched_gorder;  // [maskB*maskH*NP] all units by descending cost, or null
     const int32_t* sched_count;   // [maskB*maskH][NP][2]  entries; live tiles t0 | t1 << 16
     const int32_t* sched_entries; // [maskB*maskH][NP][KVB]
     float scale;                  // multiplies q k^T
@@ -168,6 +169,11 @@ cudaError_t launch_schedule(int QB, int KVB, int maskBH, int NP, const int32_t* 
                             int32_t* sched_count, int32_t* sched_cost, int32_t* sched_entries,
                             int32_t* sched_order, cudaStream_t stream);
 
+// The forward's units of all stored (b, h) ranked together (longest first), for masks with at
+// most this many units; larger masks rank within each (b, h) only.
+constexpr int kGlobalOrderMax = 16384;
+cudaError_t launch_global_order(int n, const int32_t* cost, int32_t* order, cudaStream_t stream);
+
 cudaError_t launch_mask_build(const MaskSpec& spec, int separate_full, int maskBH, int NP,
                               int32_t* kv_num, int32_t* kv_idx, int32_t* full_num,
                               int32_t* full_idx, int32_t* doc_stats, int32_t* sched_count,
@@ -222,6 +228,7 @@ struct fa_block_mask {
     int32_t* sched_cost;
     int32_t* sched_entries;
     int32_t* sched_order;
+    int32_t* sched_gorder;    // units of all stored (b, h) by cost, or null when too many
     int32_t* status;
     // The lists a caller reads back (fa_block_mask_get), at its block size BQ x BKV: the
     // kernel's own 128 x 128 lists when that is the block size, separate arrays otherwise.

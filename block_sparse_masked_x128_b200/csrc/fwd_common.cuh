@@ -36,23 +36,51 @@ struct Unit {
 // every (b, h), then the (r+1)-th ...) hands the longest units of the whole job out first;
 // head-major order keeps the CTAs in flight on one or two (b, h) at a time, so their K and V
 // stay in L2 when all heads' K and V together would not fit.
+// With the global ranking (sched_gorder), unit rank r of every stored (b, h) is handed out
+// for all the (b, h) that share that mask row (the broadcast copies) before rank r + 1; for a
+// fully broadcast mask that is the interleaved order.
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     const int BH = p.B * p.H;
-    int r, bh;
-    if (p.head_major) {
-        bh = u / p.NP;
-        r = u - bh * p.NP;
-    } else {
-        r = u / BH;
-        bh = u - r * BH;
-    }
-    const int b = bh / p.H, h = bh - b * p.H;
-    const int mb = (p.maskB == 1) ? 0 : b, mh = (p.maskH == 1) ? 0 : h;
-    const size_t sidx = (size_t)mb * p.maskH + mh;
+    int b, h;
+    size_t sidx;
     Unit un;
+    if (!p.head_major && p.sched_gorder) {
+        const int mult = BH / (p.maskB * p.maskH);   // (b, h) per stored mask row
+        const int rank = u / mult, k = u - rank * mult;
+        const int g = __ldg(p.sched_gorder + rank);
+        sidx = (size_t)(g / p.NP);
+        un.pair = g - (int)sidx * p.NP;
+        const int mb = (int)sidx / p.maskH, mh = (int)sidx - mb * p.maskH;
+        if (p.maskB == 1 && p.maskH == 1) {
+            b = k / p.H;
+            h = k - b * p.H;
+        } else if (p.maskB == 1) {
+            b = k;
+            h = mh;
+        } else if (p.maskH == 1) {
+            b = mb;
+            h = k;
+        } else {
+            b = mb;
+            h = mh;
+        }
+    } else {
+        int r, bh;
+        if (p.head_major) {
+            bh = u / p.NP;
+            r = u - bh * p.NP;
+        } else {
+            r = u / BH;
+            bh = u - r * BH;
+        }
+        b = bh / p.H;
+        h = bh - b * p.H;
+        const int mb = (p.maskB == 1) ? 0 : b, mh = (p.maskH == 1) ? 0 : h;
+        sidx = (size_t)mb * p.maskH + mh;
+        un.pair = __ldg(p.sched_order + sidx * p.NP + r);
+    }
     un.b = b;
     un.h = h;
-    un.pair = __ldg(p.sched_order + sidx * p.NP + r);
     FA_DCHECK_INDEX(un.pair, p.NP, p.status);
     const int2 c = __ldg(reinterpret_cast<const int2*>(p.sched_count) + sidx * p.NP + un.pair);
     un.E = c.x;

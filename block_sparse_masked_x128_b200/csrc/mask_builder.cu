@@ -596,6 +596,35 @@ cudaError_t launch_mask_build(const MaskSpec& spec, int separate_full, int maskB
     return e;
 }
 
+// All units of every stored (b, h) ranked together by descending cost (ties by index): entry r
+// is the unit index sidx * NP + pair of rank r.  One CTA; n <= kGlobalOrderMax.
+__global__ void __launch_bounds__(1024) global_order_kernel(int n, const int32_t* __restrict__ cost,
+                                                           int32_t* __restrict__ order) {
+    extern __shared__ int s_gcost[];
+    for (int i = threadIdx.x; i < n; i += blockDim.x) s_gcost[i] = cost[i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int c = s_gcost[i];
+        int rank = 0;
+        for (int o = 0; o < n; ++o) {
+            const int co = s_gcost[o];
+            rank += (co > c) || (co == c && o < i);
+        }
+        order[rank] = i;
+    }
+}
+
+cudaError_t launch_global_order(int n, const int32_t* cost, int32_t* order, cudaStream_t stream) {
+    if (n <= 0 || n > kGlobalOrderMax) return cudaErrorInvalidValue;
+    const int smem = n * (int)sizeof(int);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(global_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+    }
+    global_order_kernel<<<1, 1024, smem, stream>>>(n, cost, order);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_schedule(int QB, int KVB, int maskBH, int NP, const int32_t* kv_num,
                             const int32_t* kv_idx, const int32_t* full_num, const int32_t* full_idx,
                             int32_t* sched_count, int32_t* sched_cost, int32_t* sched_entries,
