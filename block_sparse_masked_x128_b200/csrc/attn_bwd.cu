@@ -63,9 +63,10 @@ enum : int {
     kBbAccFree = 5,     // the epilogue has read them
     kBbDrain = 6,
     kBbLoaded = 7,      // all eight math warps hold S and dP in registers
-    kBbUnitFull = 8,    // + unit-ring slot (2)
-    kBbUnitEmpty = 10,  // + unit-ring slot (2)
-    kBbSlot = 12        // + stage (full), then + stage (empty)
+    kBbAccDone = 8,     // the accumulating MMAs of the last entry are done (P, dS columns free)
+    kBbUnitFull = 9,    // + unit-ring slot (2)
+    kBbUnitEmpty = 11,  // + unit-ring slot (2)
+    kBbSlot = 13        // + stage (full), then + stage (empty)
 };
 
 // KV: the dK/dV kernel (its stages also carry 128 lse and 128 Delta values).
@@ -85,6 +86,16 @@ struct BCfg {
     static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;   // + alignment slack
     static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
+    // Where TMEM has room (the dK/dV pass at D = 64, the dQ pass at both head sizes) the 16-bit
+    // P and dS get columns of their own after the accumulators, so the next entry's S and dP can
+    // be computed while the math warps still work on the current entry; otherwise (the dK/dV
+    // pass at D = 128 fills all 512 columns) P and dS are written over the first 64 columns of
+    // S and dP, and the MMAs and the element-wise pass alternate.
+    static constexpr bool kSep = KV ? (D == 64) : true;
+    static constexpr uint32_t kAccEnd = KV ? 256 + 2 * D : 256 + D;
+    static constexpr uint32_t kColP = kSep ? kAccEnd : kColS;
+    static constexpr uint32_t kColDS = kSep ? (KV ? kAccEnd + 64 : kAccEnd) : kColDP;
+    static_assert(!kSep || kColDS + 64 <= 512, "TMEM budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -267,9 +278,21 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
             mma_ts_if(leader, tmem + dcol, tmem + acol + (uint32_t)(kk * 8), bd + (uint64_t)((kk * 2048) >> 4),
                       kIdescAcc, (kk > 0 || accumulate) ? 1u : 0u);
     };
-    uint32_t pos = 0, fix_iter = 0, acc_iter = 0, pr_iter = 0, u_iter = 0;
+    uint32_t pos = 0, fix_iter = 0, acc_iter = 0, pr_iter = 0, ld_iter = 0, u_iter = 0;
     bool ok = true;
     const uint32_t sFix0 = sbase, sFix1 = sbase + C::kTileBytes;
+    auto stage0 = [&](uint32_t ps) { return sbase + C::kStageOff + (ps % C::kStages) * C::kStageBytes; };
+    // S (or S^T) and dP (or dP^T) of the entry at ring position ps.
+    auto issue_s_dp = [&](uint32_t ps) -> bool {
+        const int s = (int)(ps % C::kStages);
+        if (!wait(C::kBarSlotFull + s, (ps / C::kStages) & 1u)) return false;
+        tc_fence_after();
+        const uint32_t st0 = stage0(ps), st1 = st0 + C::kTileBytes;
+        issue_ss(C::kColS, sFix0, st0);    // dK/dV pass: S^T = K_j Q_i^T;  dQ pass: S = Q_i K_j^T
+        issue_ss(C::kColDP, sFix1, st1);   // dK/dV pass: dP^T = V_j dO_i^T; dQ pass: dP = dO_i V_j^T
+        tc_commit_if(leader, bar(kBbSFull));
+        return true;
+    };
     for (;;) {
         const int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, ok);
         if (u < 0) break;
@@ -278,31 +301,37 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
         if (!wait(kBbFixFull, fix_iter & 1u)) { ok = false; break; }
         ++fix_iter;
         tc_fence_after();
+        if constexpr (C::kSep) {
+            if (!issue_s_dp(pos)) { ok = false; break; }
+        }
         for (int e = 0; e < un.E; ++e) {
-            const int s = (int)(pos % C::kStages);
-            if (!wait(C::kBarSlotFull + s, (pos / C::kStages) & 1u)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t st0 = sbase + C::kStageOff + (uint32_t)s * C::kStageBytes;
-            const uint32_t st1 = st0 + C::kTileBytes;
-            if constexpr (KV) {
-                issue_ss(C::kColS, sFix0, st0);    // S^T = K_j Q_i^T
-                issue_ss(C::kColDP, sFix1, st1);   // dP^T = V_j dO_i^T
+            const uint32_t ps = pos;
+            if constexpr (C::kSep) {
+                // The next entry's S and dP as soon as the math warps hold this entry's.
+                if (e + 1 < un.E) {
+                    if (!wait(kBbLoaded, ld_iter & 1u)) { ok = false; break; }
+                    ++ld_iter;
+                    if (!issue_s_dp(ps + 1)) { ok = false; break; }
+                } else {
+                    if (!wait(kBbLoaded, ld_iter & 1u)) { ok = false; break; }
+                    ++ld_iter;
+                }
             } else {
-                issue_ss(C::kColS, sFix0, st0);    // S = Q_i K_j^T
-                issue_ss(C::kColDP, sFix1, st1);   // dP = dO_i V_j^T
+                if (!issue_s_dp(ps)) { ok = false; break; }
             }
-            tc_commit_if(leader, bar(kBbSFull));
             if (!wait(kBbPReady, pr_iter & 1u)) { ok = false; break; }
             ++pr_iter;
             if (e == 0 && !wait(kBbAccFree, (acc_iter & 1u) ^ 1u)) { ok = false; break; }
             tc_fence_after();
+            const uint32_t st0 = stage0(ps), st1 = st0 + C::kTileBytes;
             if constexpr (KV) {
-                issue_ts(C::kColAcc0, C::kColS, st1, e > 0);    // dV += P^T dO_i
-                issue_ts(C::kColAcc1, C::kColDP, st0, e > 0);   // dK += dS^T Q_i
+                issue_ts(C::kColAcc0, C::kColP, st1, e > 0);    // dV += P^T dO_i
+                issue_ts(C::kColAcc1, C::kColDS, st0, e > 0);   // dK += dS^T Q_i
             } else {
-                issue_ts(C::kColAcc0, C::kColDP, st0, e > 0);   // dQ += dS K_j
+                issue_ts(C::kColAcc0, C::kColDS, st0, e > 0);   // dQ += dS K_j
             }
-            tc_commit_if(leader, bar(C::kBarSlotEmpty + s));
+            tc_commit_if(leader, bar(C::kBarSlotEmpty + (int)(ps % C::kStages)));
+            if constexpr (C::kSep) tc_commit_if(leader, bar(kBbAccDone));
             ++pos;
         }
         if (!ok) break;
@@ -354,13 +383,13 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
     const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_bits + C::kColS + 64u * g;
     const uint32_t tDP = tmem + lane_bits + C::kColDP + 64u * g;
-    const uint32_t tP = tmem + lane_bits + C::kColS + 32u * g;     // 16-bit pairs over S
-    const uint32_t tDS = tmem + lane_bits + C::kColDP + 32u * g;   // 16-bit pairs over dP
+    const uint32_t tP = tmem + lane_bits + C::kColP + 32u * g;     // 16-bit pairs
+    const uint32_t tDS = tmem + lane_bits + C::kColDS + 32u * g;
     auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
     auto wait = [&](int i, uint32_t par) {
         return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
     };
-    uint32_t pos = 0, sf_iter = 0, acc_iter = 0, u_iter = 0, ld_iter = 0;
+    uint32_t pos = 0, sf_iter = 0, acc_iter = 0, u_iter = 0, ld_iter = 0, ad_iter = 0;
     bool ok = true;
     for (;;) {
         const int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, ok);
@@ -423,11 +452,16 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
             reg_fence<32>(sr[1]);
             reg_fence<32>(dr[0]);
             reg_fence<32>(dr[1]);
-            // Both column halves are in registers before either group overwrites S or dP: a
-            // rendezvous of the eight math warps on an mbarrier (a bounded wait).
+            // S and dP are in registers: with separate P / dS columns the MMA warp may compute
+            // the next entry's into them; otherwise both column halves must be in registers
+            // before either group overwrites S or dP (a rendezvous of the eight math warps on
+            // an mbarrier, a bounded wait).
+            tc_fence_before();
             mbar_arrive_warp(bar(kBbLoaded));
-            if (!wait(kBbLoaded, ld_iter & 1u)) { ok = false; break; }
-            ++ld_iter;
+            if constexpr (!C::kSep) {
+                if (!wait(kBbLoaded, ld_iter & 1u)) { ok = false; break; }
+                ++ld_iter;
+            }
             const int col0 = t * kBlock + 64 * g;        // first column position (q or kv)
             // Live columns [lo, hi] of this row on a partial tile (+ the document compare).
             int lo = 0, hi = 63;
@@ -457,38 +491,64 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
                 vd = reinterpret_cast<const float*>(st + 512) + 64 * g;
             }
             uint32_t pk[2][16], dk[2][16];
-            // Column c's bias is slope * (kv - q): +1 per column in the dQ kernel (kv grows),
-            // -1 per column in the dK/dV kernel (q grows).
+            // Column c's bias is slope * (kv - q): +1 per column in the dQ pass (kv grows),
+            // -1 per column in the dK/dV pass (q grows).  Pairs of columns in packed f32x2.
             const float bias0 = KV ? slope_log2 * (float)(row_pos - col0) : slope_log2 * (float)(col0 - row_pos);
             const float dbias = KV ? -slope_log2 : slope_log2;
+            float2 pos2 = make_float2(bias0, bias0 + dbias);
+            const float2 step2 = make_float2(2.f * dbias, 2.f * dbias);
+            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+            const float2 inv2 = make_float2(p.inv_softcap_scale, p.inv_softcap_scale);
+            const float2 cap2 = make_float2(p.softcap_log2, p.softcap_log2);
+            const float2 nrl2 = make_float2(-row_l, -row_l), nrd2 = make_float2(-row_d, -row_d);
+            const float2 one2 = make_float2(1.f, 1.f);
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    float pv[2], dsv[2];
-#pragma unroll
-                    for (int k2 = 0; k2 < 2; ++k2) {
-                        const int c = 32 * h2 + 2 * i + k2;
-                        const float raw = __uint_as_float(sr[h2][2 * i + k2]);
-                        const float dp = __uint_as_float(dr[h2][2 * i + k2]);
-                        float th;
-                        const float x = score_log2<SCORE>(p, raw, bias0 + dbias * (float)c, th);
-                        bool live = true;
-                        if (!full) {
-                            live = c >= lo && c <= hi;
-                            if constexpr (kDoc) live = live && (__ldg(p.doc_id + col0 + c) == row_doc);
-                        }
-                        const float lq = KV ? vl[c] : row_l;
-                        const float dq = KV ? vd[c] : row_d;
-                        const float pr = live ? ex2_approx(x - lq) : 0.f;
-                        float dsr = pr * (dp - dq);
-                        if constexpr (kSoftcap) dsr *= (1.0f - th * th);
-                        pv[k2] = pr;
-                        dsv[k2] = dsr;
+                    const int c = 32 * h2 + 2 * i;
+                    const float2 raw = make_float2(__uint_as_float(sr[h2][2 * i]), __uint_as_float(sr[h2][2 * i + 1]));
+                    const float2 dp = make_float2(__uint_as_float(dr[h2][2 * i]), __uint_as_float(dr[h2][2 * i + 1]));
+                    float2 x, th;
+                    if constexpr (kSoftcap) {
+                        const float2 a = __fmul2_rn(raw, inv2);
+                        th = make_float2(tanh_approx(a.x), tanh_approx(a.y));
+                        x = __fmul2_rn(cap2, th);
+                    } else {
+                        x = __fmul2_rn(raw, sc2);
                     }
-                    pk[h2][i] = pack2<BF16>(pv[0], pv[1]);
-                    dk[h2][i] = pack2<BF16>(dsv[0], dsv[1]);
+                    if constexpr (kAlibi) {
+                        x = __fadd2_rn(x, pos2);
+                        pos2 = __fadd2_rn(pos2, step2);
+                    }
+                    float2 nl = nrl2, nd = nrd2;
+                    if constexpr (KV) {
+                        const float2 l2 = *reinterpret_cast<const float2*>(vl + c);
+                        const float2 d2 = *reinterpret_cast<const float2*>(vd + c);
+                        nl = make_float2(-l2.x, -l2.y);
+                        nd = make_float2(-d2.x, -d2.y);
+                    }
+                    const float2 ex = __fadd2_rn(x, nl);
+                    float2 pr = make_float2(ex2_approx(ex.x), ex2_approx(ex.y));
+                    if (!full) {
+                        bool l0 = c >= lo && c <= hi, l1 = c + 1 >= lo && c + 1 <= hi;
+                        if constexpr (kDoc) {
+                            l0 = l0 && (__ldg(p.doc_id + col0 + c) == row_doc);
+                            l1 = l1 && (__ldg(p.doc_id + col0 + c + 1) == row_doc);
+                        }
+                        pr = make_float2(l0 ? pr.x : 0.f, l1 ? pr.y : 0.f);
+                    }
+                    float2 ds = __fmul2_rn(pr, __fadd2_rn(dp, nd));
+                    if constexpr (kSoftcap) ds = __fmul2_rn(ds, __ffma2_rn(make_float2(-th.x, -th.y), th, one2));
+                    pk[h2][i] = pack2<BF16>(pr.x, pr.y);
+                    dk[h2][i] = pack2<BF16>(ds.x, ds.y);
                 }
+            }
+            if constexpr (C::kSep) {
+                // The last entry's accumulating MMAs read the P / dS columns: wait for them.
+                if (!wait(kBbAccDone, (ad_iter & 1u) ^ 1u)) { ok = false; break; }
+                ++ad_iter;
+                tc_fence_after();
             }
             if constexpr (KV) {
                 tmem_st_32x32b_x16(tP, pk[0]);
@@ -554,6 +614,7 @@ attn_bwd_kernel(const __grid_constant__ BwdParams p, const __grid_constant__ CUt
         mbar_init(bars + 8u * kBbAccFree, 8);
         mbar_init(bars + 8u * kBbDrain, 1);
         mbar_init(bars + 8u * kBbLoaded, 8);
+        mbar_init(bars + 8u * kBbAccDone, 1);
         for (int r = 0; r < kUnitRing; ++r) {
             mbar_init(bars + 8u * (C::kBarUFull + r), 1);
             mbar_init(bars + 8u * (C::kBarUEmpty + r), 9);   // the MMA warp + 8 math warps
