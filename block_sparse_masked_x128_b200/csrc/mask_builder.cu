@@ -78,6 +78,8 @@ __device__ __forceinline__ void interval_bounds(const MaskSpec& m, long long& lo
 __device__ int classify_fast(const MaskSpec& m, int i, int j) {
     const int qs = i * m.BQ, qe = min(qs + m.BQ, m.Q_LEN) - 1;
     const int ks = j * m.BKV, ke = min(ks + m.BKV, m.KV_LEN) - 1;
+    // A tile wholly past the context (a batch shorter than KV_LEN under kv_lens) has no key.
+    if (ks >= m.KV_LEN || qs >= m.Q_LEN) return kDead;
     const bool ragged = (qe - qs + 1 < m.BQ) || (ke - ks + 1 < m.BKV);
     long long lo, hi;
     interval_bounds(m, lo, hi);

@@ -102,9 +102,9 @@ def test_in_place_and_strided_views():
 
 def test_unsupported_shapes_and_host_buffers_are_refused():
     fa = _fa()
-    s = torch.zeros(1, 1, 4, 100, dtype=torch.bfloat16, device="cuda")
+    s = torch.zeros(1, 1, 4, 104, dtype=torch.bfloat16, device="cuda")[..., :100]   # K % 8 != 0
     with pytest.raises(fa.FaError) as e:
-        fa.masked_softmax(s)
+        fa.masked_softmax(s, out=torch.zeros(1, 1, 4, 104, dtype=torch.bfloat16, device="cuda")[..., :100])
     assert e.value.status == fa.FA_ERR_UNSUPPORTED
     s = torch.zeros(1, 1, 2, 32776, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(fa.FaError) as e:
