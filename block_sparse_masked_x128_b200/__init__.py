@@ -46,7 +46,7 @@ EXPORTED = ("fa_create_block_mask", "fa_forward", "fa_block_mask_get", "fa_get_d
             "fa_destroy_block_mask", "fa_status_string", "fa_last_error_message",
             "fa_create_block_mask_noalloc", "fa_debug_set_stall", "fa_masked_softmax",
             "fa_masked_softmax_status", "fa_backward", "fa_backward_workspace_bytes",
-            "fa_block_mask_from_kv_blocks", "fa_forward_paged")
+            "fa_block_mask_from_kv_blocks", "fa_forward_paged", "fa_forward_paged_workspace_bytes")
 
 
 class FaMaskParams(ctypes.Structure):
@@ -90,8 +90,11 @@ _lib.fa_forward.restype = _status
 _lib.fa_forward_paged.argtypes = [ctypes.POINTER(FaTensor), ctypes.POINTER(FaTensor), ctypes.POINTER(FaTensor),
                                   ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_uint32,
                                   ctypes.POINTER(FaScoreParams), ctypes.c_float, ctypes.POINTER(FaTensor),
-                                  ctypes.c_void_p, ctypes.c_void_p]
+                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
 _lib.fa_forward_paged.restype = _status
+_lib.fa_forward_paged_workspace_bytes.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                  ctypes.c_int64, ctypes.c_int64]
+_lib.fa_forward_paged_workspace_bytes.restype = ctypes.c_size_t
 _lib.fa_create_block_mask_noalloc.argtypes = [
     ctypes.c_uint32, ctypes.POINTER(FaMaskParams), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
     ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -429,10 +432,11 @@ def block_mask_from_kv_blocks(kv_num_blocks, kv_indices, full_kv_num_blocks=None
 def flex_attention(q, k, v, block_mask: BlockMask, *, score_mod: int = FA_SCORE_NONE,
                    softcap: float = 30.0, alibi_slopes=None, scale: Optional[float] = None,
                    out=None, lse=None, return_lse: bool = True, page_table=None,
-                   stream=None) -> Tuple:
+                   split_decode: bool = True, workspace=None, stream=None) -> Tuple:
     """Fused block-sparse attention forward: returns (out, lse) (lse None if not requested).
     With page_table (int32 CUDA tensor (B, n) of page indices), k and v are (n_pages, H, 128, D)
-    page pools and the mask's KV_LEN is the logical context length."""
+    page pools and the mask's KV_LEN is the logical context length; with at most 4 query rows
+    and split_decode the split decode path runs (its workspace is allocated when not given)."""
     import torch
     if out is None:
         out = torch.empty_like(q)
@@ -458,12 +462,21 @@ def flex_attention(q, k, v, block_mask: BlockMask, *, score_mod: int = FA_SCORE_
                     and page_table.device == q.device):
                 raise ValueError("page_table must be an int32 CUDA tensor (B, >= kv blocks) with "
                                  "contiguous rows on q's device")
+            ws_ptr, ws_bytes = None, 0
+            if split_decode:
+                need = int(_lib.fa_forward_paged_workspace_bytes(block_mask.handle, q.shape[0], q.shape[1],
+                                                                 q.shape[2], q.shape[3]))
+                if need > 0:
+                    if workspace is None:
+                        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+                    ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
             st = _lib.fa_forward_paged(ctypes.byref(fa_tensor(q)), ctypes.byref(fa_tensor(k)),
                                        ctypes.byref(fa_tensor(v)), page_table.data_ptr(),
                                        page_table.stride(0), block_mask.handle, int(score_mod),
                                        ctypes.byref(params), float(scale) if scale is not None else -1.0,
                                        ctypes.byref(fa_tensor(out)),
-                                       lse.data_ptr() if lse is not None else None, _stream_ptr(stream))
+                                       lse.data_ptr() if lse is not None else None, ws_ptr, ws_bytes,
+                                       _stream_ptr(stream))
             _check(st, "fa_forward_paged")
     return out, lse
 

@@ -28,7 +28,7 @@ LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libfa_b200.so")
 TRACE_LIB = os.path.join(LIBDIR, "libfa_b200_trace.so")
 DEBUG_LIB = os.path.join(LIBDIR, "libfa_b200_debug.so")
-SOURCES = ["api.cu", "mask_builder.cu", "attn_fwd.cu", "noalloc.cu", "masked_softmax.cu", "attn_bwd.cu"]
+SOURCES = ["api.cu", "mask_builder.cu", "attn_fwd.cu", "noalloc.cu", "masked_softmax.cu", "attn_bwd.cu", "decode.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

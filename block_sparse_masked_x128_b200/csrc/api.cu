@@ -569,10 +569,20 @@ namespace {
 
 // The forward of fa_forward and fa_forward_paged.  With a page table, k and v are page pools
 // (n_pages, H, 128, D) and the mask's KV_LEN is the logical context length.
+// Split decode: tiles per CTA so that about 8 CTAs per SM share the (b, h)'s tiles.
+void decode_chunking(int KVB, int64_t BH, int nsm, int& tiles_per_chunk, int& max_chunks) {
+    const int64_t target = 8 * (int64_t)(nsm > 0 ? nsm : 148);
+    const int64_t per_bh = (target + BH - 1) / BH;
+    int64_t tpc = (KVB + per_bh - 1) / per_bh;
+    if (tpc < 1) tpc = 1;
+    tiles_per_chunk = (int)tpc;
+    max_chunks = (int)((KVB + tpc - 1) / tpc);
+}
+
 fa_status_t forward_impl(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tensor_t* v,
                          const int32_t* page_table, int64_t page_stride, const fa_block_mask_t* m,
                          uint32_t score_mod_kind, const fa_score_params_t* params, float scale,
-                         fa_tensor_t* out, float* lse, void* stream) {
+                         fa_tensor_t* out, float* lse, void* stream, bool check_only = false) {
     fa_status_t s;
     if ((s = check_tensor(q, "q")) != FA_OK) return s;
     if ((s = check_tensor(k, "k")) != FA_OK) return s;
@@ -629,6 +639,7 @@ fa_status_t forward_impl(const fa_tensor_t* q, const fa_tensor_t* k, const fa_te
         return s;
     if (page_table && (s = fa::check_device_memory(page_table, dev, "page_table")) != FA_OK) return s;
 
+    if (check_only) return FA_OK;
     CUtensorMap tq, tk, tv;
     if ((s = make_tmap(&tq, q, "q")) != FA_OK) return s;
     if ((s = make_tmap(&tk, k, "k")) != FA_OK) return s;
@@ -894,17 +905,91 @@ fa_status_t fa_forward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_tens
     return forward_impl(q, k, v, nullptr, 0, m, score_mod_kind, params, scale, out, lse, stream);
 }
 
+size_t fa_forward_paged_workspace_bytes(const fa_block_mask_t* m, int64_t B, int64_t H,
+                                        int64_t Q_LEN, int64_t D) {
+    if (!m || B <= 0 || H <= 0 || Q_LEN <= 0 || Q_LEN > fa::kDecodeMaxQ || (D != 64 && D != 128) ||
+        B * H > 65535)
+        return 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    int tpc = 0, chunks = 0;
+    decode_chunking(m->KVB, B * H, sm_count(dev), tpc, chunks);
+    return (size_t)(B * H * Q_LEN) * chunks * (size_t)(D + 2) * 4;
+}
+
 fa_status_t fa_forward_paged(const fa_tensor_t* q, const fa_tensor_t* k_pages,
                              const fa_tensor_t* v_pages, const int32_t* page_table,
                              int64_t page_table_stride, const fa_block_mask_t* m,
                              uint32_t score_mod_kind, const fa_score_params_t* params, float scale,
-                             fa_tensor_t* out, float* lse, void* stream) {
+                             fa_tensor_t* out, float* lse, void* workspace, size_t workspace_bytes,
+                             void* stream) {
     NvtxRange nvtx_range("fa_forward_paged");
     if (!page_table) return fail(FA_ERR_INVALID_ARG, "page_table is NULL");
     if ((reinterpret_cast<uintptr_t>(page_table) & 3u) != 0)
         return fail(FA_ERR_INVALID_ARG, "page_table is not 4-byte aligned");
-    return forward_impl(q, k_pages, v_pages, page_table, page_table_stride, m, score_mod_kind, params,
-                        scale, out, lse, stream);
+    const bool split = workspace && q && q->S >= 1 && q->S <= fa::kDecodeMaxQ && q->B * q->H <= 65535;
+    if (!split)
+        return forward_impl(q, k_pages, v_pages, page_table, page_table_stride, m, score_mod_kind, params,
+                            scale, out, lse, stream);
+    // The split decode path: every argument check of the forward first (nothing is launched
+    // on an error), then the workspace.
+    fa_status_t s = forward_impl(q, k_pages, v_pages, page_table, page_table_stride, m, score_mod_kind,
+                                 params, scale, out, lse, stream, /*check_only=*/true);
+    if (s != FA_OK) return s;
+    if (q->B == 0 || q->H == 0) return ok();
+    const size_t need = fa_forward_paged_workspace_bytes(m, q->B, q->H, q->S, q->D);
+    if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15u))
+        return fail(FA_ERR_INVALID_ARG, "workspace must be 16-byte aligned device memory of at least %zu bytes", need);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if ((s = fa::check_device_memory(workspace, dev, "workspace")) != FA_OK) return s;
+    fa::DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = (int32_t)q->B;
+    p.H = (int32_t)q->H;
+    p.Q_LEN = (int32_t)q->S;
+    p.KV_LEN = m->KV_LEN;
+    p.KVB = m->KVB;
+    p.NP = m->NP;
+    p.maskB = m->B;
+    p.maskH = m->H;
+    p.mask_kind = m->mask_kind;
+    p.window = m->window;
+    p.doc_id = m->doc;
+    p.kv_lens = m->kv_lens;
+    p.sched_count = m->sched_count;
+    p.sched_entries = m->sched_entries;
+    p.q = q->data;
+    p.k = k_pages->data;
+    p.v = v_pages->data;
+    for (int i = 0; i < 3; ++i) {
+        p.q_stride[i] = q->stride[i];
+        p.k_stride[i] = k_pages->stride[i];
+        p.v_stride[i] = v_pages->stride[i];
+        p.out_stride[i] = out->stride[i];
+    }
+    p.page_table = page_table;
+    p.page_stride = (int32_t)page_table_stride;
+    p.n_pages = (int32_t)k_pages->B;
+    const float sc = (scale > 0.f) ? scale : (float)(1.0 / std::sqrt((double)q->D));
+    const float cap = (score_mod_kind & FA_SCORE_SOFTCAP) ? params->softcap : 1.f;
+    p.scale_log2 = sc * 1.4426950408889634f;
+    p.softcap_log2 = cap * 1.4426950408889634f;
+    p.inv_softcap_scale = sc / cap;
+    p.alibi_slopes = params ? params->alibi_slopes : nullptr;
+    p.out = out->data;
+    p.lse = lse;
+    p.partials = static_cast<float*>(workspace);
+    decode_chunking(m->KVB, q->B * q->H, sm_count(dev), p.tiles_per_chunk, p.max_chunks);
+    p.status = m->status;
+    e = fa::launch_decode(p, (int)q->D, q->dtype == FA_DTYPE_BF16, (int)score_mod_kind,
+                          static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return ok();
 }
 
 // Test hook for failure detection (see the header): read by every later fa_forward.

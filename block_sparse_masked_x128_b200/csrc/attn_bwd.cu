@@ -429,7 +429,7 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
             row_d = __ldg(p.delta + vec_row + row_pos);
         }
         const int row_doc = (kDoc && row_pos < p.QB * kBlock) ? __ldg(p.doc_id + row_pos) : 0;
-        const int kv_len = p.kv_lens ? min(p.KV_LEN, __ldg(p.kv_lens + un.b)) : p.KV_LEN;
+        const int kv_len = p.kv_lens ? min(p.KV_LEN, __ldg(p.kv_lens + (p.maskB == 1 ? 0 : un.b))) : p.KV_LEN;
         EntryReader er;
         er.init(un.entries, un.E);
         for (int e = 0; e < un.E; ++e) {

@@ -343,7 +343,7 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
             continue;
         }
         const int q = qblk * kBlock + row;
-        const int kv_len = p.kv_lens ? min(p.KV_LEN, __ldg(p.kv_lens + un.b)) : p.KV_LEN;
+        const int kv_len = p.kv_lens ? min(p.KV_LEN, __ldg(p.kv_lens + (p.maskB == 1 ? 0 : un.b))) : p.KV_LEN;
         float slope_log2 = 0.f;
         if constexpr (has_alibi) {
             float slope;

@@ -142,6 +142,33 @@ struct BwdParams {
     int32_t* sched_ctr;
 };
 
+// Parameters of the split decode path (decode.cu): Q_LEN <= 4 query rows over paged K/V.
+struct DecodeParams {
+    int32_t B, H, Q_LEN, KV_LEN, KVB, NP, maskB, maskH;
+    uint32_t mask_kind;
+    int32_t window;
+    const int32_t* doc_id;
+    const int32_t* kv_lens;
+    const int32_t* sched_count;   // the block mask's forward schedule (query block 0 of each pair)
+    const int32_t* sched_entries;
+    const void* q;
+    const void* k;                // page pools (n_pages, H, 128, D)
+    const void* v;
+    int64_t q_stride[3], k_stride[3], v_stride[3];
+    const int32_t* page_table;
+    int32_t page_stride, n_pages;
+    float scale_log2, softcap_log2, inv_softcap_scale;
+    const float* alibi_slopes;
+    void* out;
+    int64_t out_stride[3];
+    float* lse;
+    float* partials;              // workspace [B*H][Q_LEN][max_chunks][D + 2]: m, l, O
+    int32_t max_chunks, tiles_per_chunk;
+    int32_t* status;
+};
+constexpr int kDecodeMaxQ = 4;
+cudaError_t launch_decode(const DecodeParams& p, int D, bool bf16, int score_kind, cudaStream_t st);
+
 cudaError_t launch_bwd_preprocess(const void* out, const int64_t out_stride[3], const void* dout,
                                   const int64_t dout_stride[3], const float* lse, int B, int H,
                                   int Q_LEN, int q_pad, int D, bool bf16, float* lse_log2,

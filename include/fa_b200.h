@@ -258,14 +258,24 @@ fa_status_t fa_create_block_mask_noalloc(uint32_t mask_kind, const fa_mask_param
  *                      kv_blocks; only the entries of listed tiles are read
  *   block_mask         built for the logical lengths Q_LEN x KV_LEN (usually with kv_lens,
  *                      one context length per batch element, and no mask kind for decode)
- * Everything else is fa_forward's.  A page index outside [0, n_pages) reads as zeros and is
- * recorded: fa_get_device_status then returns FA_ERR_INVALID_ARG.
+ *   workspace          NULL, or device scratch of fa_forward_paged_workspace_bytes(block_mask,
+ *                      B, H, Q_LEN, D) bytes, 16-byte aligned, caller-owned.  With Q_LEN <= 4 and
+ *                      a workspace the call runs the split decode path: each (b, h)'s pages are
+ *                      shared out to several CTAs on the CUDA cores (the work is reading K and
+ *                      V once), whose partial results a second kernel merges; otherwise the
+ *                      tensor-core forward runs.  Calls that overlap need distinct workspaces.
+ * Everything else is fa_forward's.  A page index outside [0, n_pages) reads as zeros (the
+ * split path skips the page) and is recorded: fa_get_device_status then returns
+ * FA_ERR_INVALID_ARG.
  */
+size_t fa_forward_paged_workspace_bytes(const fa_block_mask_t* block_mask, int64_t B, int64_t H,
+                                        int64_t Q_LEN, int64_t D);   /* 0: no split path */
 fa_status_t fa_forward_paged(const fa_tensor_t* q, const fa_tensor_t* k_pages,
                              const fa_tensor_t* v_pages, const int32_t* page_table,
                              int64_t page_table_stride, const fa_block_mask_t* block_mask,
                              uint32_t score_mod_kind, const fa_score_params_t* params, float scale,
-                             fa_tensor_t* out, float* lse, void* stream);
+                             fa_tensor_t* out, float* lse, void* workspace, size_t workspace_bytes,
+                             void* stream);
 
 /*
  * fa_backward -- gradients of fa_forward over the same block mask, deterministic.

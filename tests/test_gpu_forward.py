@@ -377,23 +377,31 @@ def test_per_batch_sequence_lengths():
     compare(out, lse, O, L)
 
 
-@pytest.mark.parametrize("Q", [1, 5])
-def test_paged_decode_equals_contiguous_and_the_oracle(Q):
-    # PagedAttention through block indices: K/V in shuffled 128-token pages of one pool.
+@pytest.mark.parametrize("Q,D,dtype,score", [(1, 128, "bf16", 0), (3, 64, "fp16", 0), (1, 128, "bf16", 3),
+                                             (4, 64, "bf16", 2), (5, 128, "bf16", 0)])
+def test_paged_decode_matches_contiguous_and_the_oracle(Q, D, dtype, score):
+    # PagedAttention through block indices: K/V in shuffled 128-token pages of one pool.  Up to
+    # 4 query rows run the split decode path (checked against the oracle); the tensor-core path
+    # over the pages (split_decode=False, and always for more rows) equals the contiguous
+    # forward bit for bit.
     fa = fa_module()
-    dw = wl.DecodeWorkload("decode_small", B=4, H=4, D=128, lo=130, hi=2500, Q=Q, seed=30)
+    dw = wl.DecodeWorkload("decode_small", B=4, H=4, D=D, lo=130, hi=2500, Q=Q, dtype=dtype, seed=30)
     q, k, v, kp, vp, table, lens = wl.make_decode(dw)
     KV = k.shape[2]
     lens_t = torch.from_numpy(lens).cuda()
     bm = fa.create_block_mask(0, dw.B, None, Q, KV, kv_lens=lens_t)
-    paged = fa.flex_attention(q.cuda(), kp.cuda(), vp.cuda(), bm, page_table=table.cuda())
-    contig = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm)
+    qd, kd, vd, kpd, vpd, td = (t.cuda() for t in (q, k, v, kp, vp, table))
+    split = fa.flex_attention(qd, kpd, vpd, bm, page_table=td, score_mod=score, softcap=20.0)
+    tc = fa.flex_attention(qd, kpd, vpd, bm, page_table=td, score_mod=score, softcap=20.0, split_decode=False)
+    contig = fa.flex_attention(qd, kd, vd, bm, score_mod=score, softcap=20.0)
     torch.cuda.synchronize()
     assert bm.device_status() == fa.FA_OK
-    assert torch.equal(paged[0], contig[0]) and torch.equal(paged[1], contig[1])
+    assert torch.equal(tc[0], contig[0]) and torch.equal(tc[1], contig[1])
     mm = oracle.make_mask_mod(0, kv_lens=lens)
-    O, L = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), mm, None, scale=dw.scale)
-    compare(paged[0], paged[1], O, L)
+    sm = oracle.make_score_mod(score, H=dw.H, softcap=20.0)
+    O, L = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), mm, sm, scale=dw.scale)
+    compare(split[0], split[1], O, L)
+    compare(tc[0], tc[1], O, L)
 
 
 def test_paged_page_out_of_range_is_reported():
