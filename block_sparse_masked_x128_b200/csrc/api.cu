@@ -804,6 +804,7 @@ fa_status_t fa_backward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_ten
     p.delta = delta;
     p.q_pad = q_pad;
     p.status = m->status;
+    p.stall_loads = g_stall_loads.load(std::memory_order_relaxed);
     fa_block_mask_t* mm = const_cast<fa_block_mask_t*>(m);
 
     // dK, dV: one unit per kv block; Q and dO stream, so order by head when they outgrow L2.
@@ -883,6 +884,7 @@ fa_status_t fa_masked_softmax(const fa_tensor_t* scores, uint32_t mask_kind, int
                                           (int)scores->B, (int)scores->H, (int)scores->S, (int)K,
                                           offset, mask_kind == FA_MASK_CAUSAL,
                                           scores->dtype == FA_DTYPE_BF16, nsm,
+                                          g_stall_loads.load(std::memory_order_relaxed),
                                           static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "masked-softmax launch");
     return ok();

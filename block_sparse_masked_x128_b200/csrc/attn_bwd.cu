@@ -206,6 +206,11 @@ __device__ void bwd_producer(const BwdParams& p, const CUtensorMap* tq, const CU
                            un.idx * kBlock, un.h, un.b);
         }
         ++fix_iter;
+        if (p.stall_loads) {   // test hook: let the fixed tiles land, then load nothing more
+            drain_wait(bar(kBbFixFull), (fix_iter - 1) & 1u);
+            finish();
+            return;
+        }
         EntryReader er;
         er.init(un.entries, un.E);
         const size_t vec_row = ((size_t)un.b * p.H + un.h) * (size_t)p.q_pad;

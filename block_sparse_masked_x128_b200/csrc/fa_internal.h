@@ -140,6 +140,7 @@ struct BwdParams {
     int64_t grad1_stride[3];
     int32_t* status;
     int32_t* sched_ctr;
+    int32_t stall_loads;          // test hook: the TMA warp stops after the first unit's fixed tiles
 };
 
 // Parameters of the split decode path (decode.cu): Q_LEN <= 4 query rows over paged K/V.
@@ -227,7 +228,7 @@ int masked_softmax_max_keys();
 cudaError_t launch_masked_softmax_checked(const void* in, void* out, const int64_t in_stride[3],
                                           const int64_t out_stride[3], int B, int H, int Q, int K,
                                           int64_t offset, bool causal, bool bf16, int num_sms,
-                                          cudaStream_t stream);
+                                          int stall_loads, cudaStream_t stream);
 cudaError_t masked_softmax_status(cudaStream_t stream, int32_t* out);
 
 // Counter pairs per mask for the forward's run-time unit hand-out: each launch takes the

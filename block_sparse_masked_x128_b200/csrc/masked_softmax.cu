@@ -11,15 +11,14 @@
 //
 // Organisation (HBM-bound; one persistent CTA of 512 threads per SM):
 //   * rows (b, h, q) are dealt round robin to the CTAs;
-//   * thread 0 stages each row's live prefix into shared memory with one cp.async.bulk load,
-//     a ring of `stages` row buffers deep (so up to stages - 1 rows are in flight while one
-//     is computed), completing on one mbarrier per buffer;
-//   * all threads then hold the row in registers (thread t owns the 16-byte vectors
-//     t, t + 512, ...), take the row max and the row sum of e = 2^((x - max) log2 e) with
-//     warp shuffles and a fixed-order cross-warp step, and write p = e / sum back over the
-//     buffer as 16-bit values;
-//   * thread 0 writes the row out with one cp.async.bulk store; the buffer is reloaded once
-//     that store has read it (bulk wait_group.read, one row behind).
+//   * warp 0 only moves data: it stages each row's live prefix into shared memory with one
+//     cp.async.bulk load into a ring of `stages` row buffers (completing on the buffer's
+//     `full` mbarrier), stores each computed row with one cp.async.bulk store, and as soon as
+//     that store has read the buffer, loads the row `stages` ahead into it;
+//   * warps 1-15 hold the row in registers (thread c owns the 16-byte vectors c, c + 480,
+//     ...), take the row max and the row sum of e = 2^((x - max) log2 e) with warp shuffles
+//     and a fixed-order cross-warp step on a named barrier of their own, write p = e / sum
+//     back over the buffer as 16-bit values and arrive on the buffer's `done` mbarrier.
 // Every reduction has the same order in the masked and the unmasked run, which is what
 // makes them bit-identical.  Waits are bounded: a wait that runs out sets the status word,
 // and the CTA drains its own copies before it returns.
@@ -44,12 +43,14 @@ struct SoftmaxParams {
     int32_t stages;
     uint32_t stage_bytes;   // K * 2 rounded up to 128
     int32_t* status;
+    int32_t stall_loads;    // test hook: the producer loads the first buffers only
 };
 
 namespace {
 
 constexpr int kSmThreads = 512;
 constexpr int kSmWarps = kSmThreads / 32;
+constexpr int kSmCompute = kSmThreads - 32;   // warp 0 moves data, warps 1.. compute
 constexpr uint64_t kSmWaitLimitNs = 2000000000ull;
 constexpr float kSmLog2e = 1.4426950408889634f;
 
@@ -99,17 +100,29 @@ __device__ __forceinline__ void issue_row_load(const SoftmaxParams& p, int64_t r
         bulk_load(dst, p.in + b * p.in_stride[0] + h * p.in_stride[1] + q * p.in_stride[2], bytes, bar);
 }
 
-// Bounded wait by every thread; the outcome is made block-uniform.
-__device__ __forceinline__ bool block_wait(uint32_t bar, uint32_t parity) {
-    bool ok = mbar_try_wait(bar, parity);
-    if (!ok) {
-        const uint64_t t0 = global_timer_ns();
-        for (uint32_t it = 1;; ++it) {
-            if (mbar_try_wait(bar, parity)) { ok = true; break; }
-            if ((it & 127u) == 0u && global_timer_ns() - t0 > kSmWaitLimitNs) break;
-        }
+// Bounded wait on an mbarrier phase by the calling thread.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 127u) == 0u && global_timer_ns() - t0 > kSmWaitLimitNs) return false;
     }
-    return __syncthreads_and(ok ? 1 : 0) != 0;
+}
+
+// The compute warps' barrier (named barrier 1; warp 0 never takes part), with the AND of `v`.
+__device__ __forceinline__ bool compute_bar_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(v ? 1u : 0u), "n"(kSmCompute)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void compute_bar() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kSmCompute) : "memory");
 }
 
 template <bool BF16, int VPT>
@@ -118,33 +131,88 @@ __global__ void __launch_bounds__(kSmThreads, 1) masked_softmax_kernel(const __g
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                                ~static_cast<uintptr_t>(127));
     const uint32_t sbase = smem_u32(smem);
+    // Barriers: full[s] (the row's bulk load landed), done[s] (the compute warps wrote p).
     const uint32_t bars = sbase + (uint32_t)p.stages * p.stage_bytes;
-    float* red = reinterpret_cast<float*>(smem + (size_t)p.stages * p.stage_bytes + 8 * p.stages);
+    auto full_bar = [&](int s) { return bars + 8u * (uint32_t)s; };
+    auto done_bar = [&](int s) { return bars + 8u * (uint32_t)(p.stages + s); };
+    float* red = reinterpret_cast<float*>(smem + (size_t)p.stages * p.stage_bytes + 16 * p.stages);
     float* red_max = red;
     float* red_sum = red + kSmWarps;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t grid = gridDim.x;
 
     if (tid == 0) {
-        for (int s = 0; s < p.stages; ++s) mbar_init(bars + 8u * s, 1);
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(done_bar(s), kSmCompute / 32);   // one arrival per compute warp
+        }
         fence_mbar_init();
     }
     __syncthreads();
     // Rows of this CTA: blockIdx.x + k * grid, k = 0, 1, ...; row k lives in buffer k % stages.
     const int64_t my_rows = (p.rows > blockIdx.x) ? (p.rows - blockIdx.x + grid - 1) / grid : 0;
-    int64_t issued = 0;   // rows whose load thread 0 has issued
-    if (tid == 0) {
-        for (; issued < my_rows && issued < p.stages; ++issued)
-            issue_row_load(p, blockIdx.x + issued * grid, sbase + (uint32_t)issued * p.stage_bytes,
-                           bars + 8u * (uint32_t)issued);
+
+    if (warp == 0) {
+        // Producer: loads rows ahead into free buffers; stores each computed row, and once the
+        // store has read its buffer, loads the row `stages` ahead into it.
+        if (lane == 0) {
+            int64_t issued = 0;
+            for (; issued < my_rows && issued < p.stages; ++issued)
+                issue_row_load(p, blockIdx.x + issued * grid, sbase + (uint32_t)issued * p.stage_bytes,
+                               full_bar((int)issued));
+            int64_t k = 0;
+            bool ok = true;
+            if (p.stall_loads) {   // test hook: the compute warps' wait for row `stages` runs out
+                for (int64_t kk = 0; kk < issued; ++kk) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(full_bar((int)kk), 0u) && global_timer_ns() - t0 < kSmWaitLimitNs) {
+                    }
+                }
+                k = my_rows;   // store nothing
+            }
+            for (; k < my_rows; ++k) {
+                const int s = (int)(k % p.stages);
+                if (!wait_bounded(done_bar(s), (uint32_t)((k / p.stages) & 1))) { ok = false; break; }
+                int64_t b, h, q;
+                row_coords(p, blockIdx.x + k * grid, b, h, q);
+                bulk_store(p.out + b * p.out_stride[0] + h * p.out_stride[1] + q * p.out_stride[2],
+                           sbase + (uint32_t)s * p.stage_bytes, (uint32_t)(p.K * 2));
+                bulk_commit();
+                if (issued < my_rows) {
+                    bulk_wait_read<0>();
+                    fence_proxy_async_smem();
+                    issue_row_load(p, blockIdx.x + issued * grid, sbase + (uint32_t)s * p.stage_bytes,
+                                   full_bar(s));
+                    ++issued;
+                }
+            }
+            if (!ok) {
+                atomicExch(p.status, 1);
+                // Let the loads already issued land before the CTA's shared memory goes away.
+                for (int64_t kk = k; kk < issued; ++kk) {
+                    const uint32_t bar = full_bar((int)(kk % p.stages));
+                    const uint32_t par = (uint32_t)((kk / p.stages) & 1);
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar, par) && global_timer_ns() - t0 < kSmWaitLimitNs) {
+                    }
+                }
+            }
+            bulk_wait_all();
+        }
+        __syncwarp();
+        return;
     }
+
+    // Compute warps 1 .. kSmWarps-1: thread c = tid - 32 owns the 16-byte vectors c, c + kSmCompute, ...
+    const int c = tid - 32, cw = warp - 1;
     const float kMasked = dtype_min<BF16>();
-    int64_t k = 0;
-    bool ok = true;
-    for (; k < my_rows; ++k) {
+    for (int64_t k = 0; k < my_rows; ++k) {
         const int s = (int)(k % p.stages);
-        const uint32_t buf = sbase + (uint32_t)s * p.stage_bytes;
-        if (!block_wait(bars + 8u * s, (uint32_t)((k / p.stages) & 1))) { ok = false; break; }
+        const bool landed = wait_bounded(full_bar(s), (uint32_t)((k / p.stages) & 1));
+        if (!compute_bar_and(landed)) {
+            if (c == 0) atomicExch(p.status, 1);
+            return;
+        }
         const int64_t r = blockIdx.x + k * grid;
         int64_t b, h, q;
         row_coords(p, r, b, h, q);
@@ -156,7 +224,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) masked_softmax_kernel(const __g
         float m = -INFINITY;
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-            const int64_t e0 = 8ll * (tid + kSmThreads * j);
+            const int64_t e0 = 8ll * (c + kSmCompute * j);
             if (e0 >= p.K) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) x[8 * j + i] = -INFINITY;   // past the row: no key
@@ -177,11 +245,11 @@ __global__ void __launch_bounds__(kSmThreads, 1) masked_softmax_kernel(const __g
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
-        if (lane == 0) red_max[warp] = m;
-        __syncthreads();
+        if (lane == 0) red_max[cw] = m;
+        compute_bar();
         m = red_max[0];
 #pragma unroll
-        for (int w = 1; w < kSmWarps; ++w) m = fmaxf(m, red_max[w]);
+        for (int w = 1; w < kSmCompute / 32; ++w) m = fmaxf(m, red_max[w]);
 
         // Pass 2: e = 2^((x - m) log2 e) and the row sum, in a fixed order.  A vector wholly
         // past the causal boundary holds exp(finfo.min - m) = 0 unless the whole row is
@@ -189,7 +257,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) masked_softmax_kernel(const __g
         float sum = 0.f;
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-            const int64_t e0 = 8ll * (tid + kSmThreads * j);
+            const int64_t e0 = 8ll * (c + kSmCompute * j);
             if (e0 >= p.K) continue;
             if (e0 >= n_live && m != kMasked) {
 #pragma unroll
@@ -205,18 +273,18 @@ __global__ void __launch_bounds__(kSmThreads, 1) masked_softmax_kernel(const __g
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o);
-        if (lane == 0) red_sum[warp] = sum;
-        __syncthreads();
+        if (lane == 0) red_sum[cw] = sum;
+        compute_bar();
         sum = red_sum[0];
 #pragma unroll
-        for (int w = 1; w < kSmWarps; ++w) sum += red_sum[w];
+        for (int w = 1; w < kSmCompute / 32; ++w) sum += red_sum[w];
         const float inv = 1.0f / sum;
 
-        // Pass 3: p = e / sum as 16-bit values over the buffer, then one bulk store.
+        // Pass 3: p = e / sum as 16-bit values over the buffer; the producer stores it.
         uint16_t* wrow = reinterpret_cast<uint16_t*>(smem + (size_t)s * p.stage_bytes);
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-            const int64_t e0 = 8ll * (tid + kSmThreads * j);
+            const int64_t e0 = 8ll * (c + kSmCompute * j);
             if (e0 >= p.K) continue;
             uint32_t w[4];
 #pragma unroll
@@ -224,35 +292,9 @@ __global__ void __launch_bounds__(kSmThreads, 1) masked_softmax_kernel(const __g
             *reinterpret_cast<uint4*>(wrow + e0) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            bulk_store(p.out + b * p.out_stride[0] + h * p.out_stride[1] + q * p.out_stride[2], buf,
-                       (uint32_t)(p.K * 2));
-            bulk_commit();
-            // Refill the buffer of the previous row once its store has read it.
-            if (k >= 1 && issued < my_rows) {
-                bulk_wait_read<1>();
-                fence_proxy_async_smem();
-                const int ps = (int)((k - 1) % p.stages);
-                issue_row_load(p, blockIdx.x + issued * grid, sbase + (uint32_t)ps * p.stage_bytes,
-                               bars + 8u * (uint32_t)ps);
-                ++issued;
-            }
-        }
-    }
-    if (tid == 0) {
-        if (!ok) {
-            atomicExch(p.status, 1);
-            // Let the loads already issued land before the CTA's shared memory goes away.
-            for (int64_t kk = k; kk < issued; ++kk) {
-                const uint32_t bar = bars + 8u * (uint32_t)(kk % p.stages);
-                const uint32_t par = (uint32_t)((kk / p.stages) & 1);
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(bar, par) && global_timer_ns() - t0 < kSmWaitLimitNs) {
-                }
-            }
-        }
-        bulk_wait_all();
+        mbar_arrive_warp(done_bar(s));
+        // The next row's max reduction reuses red_max only after every warp read this one's
+        // sum (they all passed the barrier above before any can pass the next one).
     }
 }
 
@@ -267,7 +309,7 @@ cudaError_t launch_t(const SoftmaxParams& p, int grid, size_t smem, cudaStream_t
 
 }  // namespace
 
-int masked_softmax_max_keys() { return kSmThreads * 8 * 8; }
+int masked_softmax_max_keys() { return 32768; }
 
 cudaError_t launch_masked_softmax(SoftmaxParams p, bool bf16, int num_sms, cudaStream_t stream) {
     // Row buffers: as many as fit in 200 KiB, 2 to 8.
@@ -282,17 +324,18 @@ cudaError_t launch_masked_softmax(SoftmaxParams p, bool bf16, int num_sms, cudaS
         if (e != cudaSuccess) return e;
         p.status = static_cast<int32_t*>(addr);
     }
-    const size_t smem = 128 + (size_t)stages * p.stage_bytes + 8 * stages + 2 * kSmWarps * sizeof(float);
+    const size_t smem = 128 + (size_t)stages * p.stage_bytes + 16 * stages + 2 * kSmWarps * sizeof(float);
     const int grid = (int)(p.rows < num_sms ? p.rows : num_sms);
-    const int vpt_needed = (p.K + 8 * kSmThreads - 1) / (8 * kSmThreads);
+    const int vpt_needed = (p.K + 8 * kSmCompute - 1) / (8 * kSmCompute);
 #define FA_SM_CASE(V)                                                              \
     if (vpt_needed <= V)                                                           \
         return bf16 ? launch_t<true, V>(p, grid, smem, stream)                     \
                     : launch_t<false, V>(p, grid, smem, stream);
     FA_SM_CASE(1)
     FA_SM_CASE(2)
-    FA_SM_CASE(4)
-    FA_SM_CASE(8)
+    FA_SM_CASE(3)
+    FA_SM_CASE(5)
+    FA_SM_CASE(9)
 #undef FA_SM_CASE
     return cudaErrorInvalidValue;
 }
@@ -300,8 +343,9 @@ cudaError_t launch_masked_softmax(SoftmaxParams p, bool bf16, int num_sms, cudaS
 cudaError_t launch_masked_softmax_checked(const void* in, void* out, const int64_t in_stride[3],
                                           const int64_t out_stride[3], int B, int H, int Q, int K,
                                           int64_t offset, bool causal, bool bf16, int num_sms,
-                                          cudaStream_t stream) {
+                                          int stall_loads, cudaStream_t stream) {
     SoftmaxParams p;
+    p.stall_loads = stall_loads;
     p.in = static_cast<const uint16_t*>(in);
     p.out = static_cast<uint16_t*>(out);
     for (int i = 0; i < 3; ++i) {

@@ -366,10 +366,12 @@ const char* fa_last_error_message(void);
 
 /*
  * Test hook for failure detection (no counterpart on the pages).  While `enable` is nonzero,
- * the TMA warp of every fa_forward launched afterwards (process-wide) loads only the first
- * query tiles and then stops, so the MMA warp's bounded wait for K runs past its limit
- * (about two seconds), every role of the kernel unwinds and releases its tensor memory,
- * and the mask's status word is set: fa_get_device_status then returns FA_ERR_TIMEOUT.
+ * the data-moving warp of every kernel launched afterwards (process-wide) stops early: the
+ * forward's TMA warp after the first query tiles, the backward's after the first unit's fixed
+ * tiles, fa_masked_softmax's producer after its first row buffers.  A bounded wait then runs
+ * past its limit (about two seconds), every role of the kernel unwinds and releases its tensor
+ * memory, and the status word is set: fa_get_device_status (fa_masked_softmax_status for the
+ * softmax) then returns FA_ERR_TIMEOUT.
  * The outputs of such a call are unspecified.  Pass 0 to restore normal operation.  Process
  * global state: not for use while other threads launch forwards.  Returns FA_OK.
  */

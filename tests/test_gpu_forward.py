@@ -55,6 +55,23 @@ def test_forward_full_size_sampled_rows(w):
     compare(out, lse, O, L, rows=rows)
 
 
+@pytest.mark.parametrize("w", wl.WORKLOADS, ids=[w.name for w in wl.WORKLOADS])
+def test_forward_full_size_one_whole_slice(w):
+    # Every row of one (b, h) slice at the workload's full size, in the launch configuration
+    # the benchmark times (all heads run; the last (b, h) is compared): a schedule or counter
+    # error confined to a few units would show here even where sampled rows miss it.
+    q, k, v, doc = workload_inputs(w)
+    out, lse, _ = run_gpu(w, q, k, v, doc)
+    b, h = w.B - 1, w.H - 1
+    sl = (slice(b, b + 1), slice(h, h + 1))
+    mm = oracle.make_mask_mod(w.mask_kind, window=w.window or None, document_id=doc)
+    sm0 = oracle.make_score_mod(w.score_kind, H=w.H, softcap=w.softcap or 30.0)
+    sm = (lambda s, bb, hh, qi, ki: sm0(s, bb, h, qi, ki)) if sm0 else None
+    O, L = oracle.attention(q[sl].float().numpy(), k[sl].float().numpy(), v[sl].float().numpy(), mm, sm,
+                            scale=w.scale)
+    compare(out[sl], lse[sl], O, L)
+
+
 @pytest.mark.parametrize("D,dtype", [(64, torch.float16), (64, torch.bfloat16), (128, torch.bfloat16),
                                      (128, torch.float16)])
 def test_window_one_returns_v_exactly(D, dtype):

@@ -38,3 +38,46 @@ def test_stalled_loads_time_out_and_the_context_survives(D):
     assert bm.device_status() == fa.FA_OK
     O, L = run_oracle(w, q, k, v)
     compare(out, lse, O, L)
+
+
+def test_stalled_backward_times_out_and_the_context_survives():
+    fa = fa_module()
+    w = wl.Workload("timeout_bwd", B=1, H=2, S=512, D=64, dtype="bf16", mask_kind=wl.MASK_CAUSAL, seed=32)
+    q, k, v = (t.cuda() for t in wl.make_qkv(w))
+    do = wl.make_dout(w).cuda()
+    bm = gpu_block_mask(wl.MASK_CAUSAL, None, None, 512, 512)
+    out, lse = fa.flex_attention(q, k, v, bm)
+    ref = fa.flex_attention_backward(q, k, v, out, lse, do, bm)
+    torch.cuda.synchronize()
+    assert bm.device_status() == fa.FA_OK
+    fa.fa_debug_set_stall(True)
+    try:
+        fa.flex_attention_backward(q, k, v, out, lse, do, bm)
+        status = bm.device_status()
+    finally:
+        fa.fa_debug_set_stall(False)
+    assert status == fa.FA_ERR_TIMEOUT
+    again = fa.flex_attention_backward(q, k, v, out, lse, do, bm)
+    torch.cuda.synchronize()
+    assert bm.device_status() == fa.FA_OK
+    assert all(torch.equal(a, b) for a, b in zip(again, ref))
+
+
+def test_stalled_masked_softmax_times_out_and_the_context_survives():
+    fa = fa_module()
+    g = torch.Generator().manual_seed(33)
+    s = torch.randn(1, 2, 1024, 4096, generator=g).to(torch.bfloat16).cuda()   # > 8 rows per CTA
+    ref = fa.masked_softmax(s)
+    torch.cuda.synchronize()
+    assert fa.fa_masked_softmax_status() == fa.FA_OK
+    fa.fa_debug_set_stall(True)
+    try:
+        fa.masked_softmax(s)
+        status = fa.fa_masked_softmax_status()
+    finally:
+        fa.fa_debug_set_stall(False)
+    assert status == fa.FA_ERR_TIMEOUT
+    assert fa.fa_masked_softmax_status() == fa.FA_OK
+    again = fa.masked_softmax(s)
+    torch.cuda.synchronize()
+    assert torch.equal(again, ref)
