@@ -89,8 +89,9 @@ struct BCfg {
     // Where TMEM has room (the dK/dV pass at D = 64, the dQ pass at both head sizes) the 16-bit
     // P and dS get columns of their own after the accumulators, so the next entry's S and dP can
     // be computed while the math warps still work on the current entry; otherwise (the dK/dV
-    // pass at D = 128 fills all 512 columns) P and dS are written over the first 64 columns of
-    // S and dP, and the MMAs and the element-wise pass alternate.
+    // pass at D = 128 fills all 512 columns) each math group writes its 16-bit P and dS over the
+    // first 32 columns of its own 64 S and dP columns (group g: 64g.., 128 + 64g..), and the
+    // MMAs and the element-wise pass alternate.
     static constexpr bool kSep = KV ? (D == 64) : true;
     static constexpr uint32_t kAccEnd = KV ? 256 + 2 * D : 256 + D;
     static constexpr uint32_t kColP = kSep ? kAccEnd : kColS;
@@ -276,12 +277,16 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
         }
     };
     // D[128 x D] (+)= A[128 x 128] B[128 x D]: A 16-bit pairs in TMEM, B MN-major in smem.
+    // The K step kk covers columns 16kk .. 16kk+15 of the 128 x 128 tile, 8 columns of 16-bit
+    // pairs: contiguous with separate P / dS columns, else in the two groups' own column blocks.
     auto issue_ts = [&](uint32_t dcol, uint32_t acol, uint32_t b, bool accumulate) {
         const uint64_t bd = make_sdesc_sw128(b, 16384, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts_if(leader, tmem + dcol, tmem + acol + (uint32_t)(kk * 8), bd + (uint64_t)((kk * 2048) >> 4),
+        for (int kk = 0; kk < kBlock / 16; ++kk) {
+            const uint32_t aoff = C::kSep ? (uint32_t)(kk * 8) : (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8);
+            mma_ts_if(leader, tmem + dcol, tmem + acol + aoff, bd + (uint64_t)((kk * 2048) >> 4),
                       kIdescAcc, (kk > 0 || accumulate) ? 1u : 0u);
+        }
     };
     uint32_t pos = 0, fix_iter = 0, acc_iter = 0, pr_iter = 0, ld_iter = 0, u_iter = 0;
     bool ok = true;
@@ -388,8 +393,10 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
     const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_bits + C::kColS + 64u * g;
     const uint32_t tDP = tmem + lane_bits + C::kColDP + 64u * g;
-    const uint32_t tP = tmem + lane_bits + C::kColP + 32u * g;     // 16-bit pairs
-    const uint32_t tDS = tmem + lane_bits + C::kColDS + 32u * g;
+    // 16-bit pairs of P and dS: 32 columns per group, after the accumulators or over the
+    // group's own S and dP columns.
+    const uint32_t tP = tmem + lane_bits + C::kColP + (C::kSep ? 32u : 64u) * g;
+    const uint32_t tDS = tmem + lane_bits + C::kColDS + (C::kSep ? 32u : 64u) * g;
     auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
     auto wait = [&](int i, uint32_t par) {
         return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
@@ -447,26 +454,6 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
             if (!wait(kBbSFull, sf_iter & 1u)) { ok = false; break; }
             ++sf_iter;
             tc_fence_after();
-            uint32_t sr[2][32], dr[2][32];
-            tmem_ld_32x32b_x32(tS, sr[0]);
-            tmem_ld_32x32b_x32(tS + 32, sr[1]);
-            tmem_ld_32x32b_x32(tDP, dr[0]);
-            tmem_ld_32x32b_x32(tDP + 32, dr[1]);
-            tmem_ld_wait();
-            reg_fence<32>(sr[0]);
-            reg_fence<32>(sr[1]);
-            reg_fence<32>(dr[0]);
-            reg_fence<32>(dr[1]);
-            // S and dP are in registers: with separate P / dS columns the MMA warp may compute
-            // the next entry's into them; otherwise both column halves must be in registers
-            // before either group overwrites S or dP (a rendezvous of the eight math warps on
-            // an mbarrier, a bounded wait).
-            tc_fence_before();
-            mbar_arrive_warp(bar(kBbLoaded));
-            if constexpr (!C::kSep) {
-                if (!wait(kBbLoaded, ld_iter & 1u)) { ok = false; break; }
-                ++ld_iter;
-            }
             const int col0 = t * kBlock + 64 * g;        // first column position (q or kv)
             // Live columns [lo, hi] of this row on a partial tile (+ the document compare).
             int lo = 0, hi = 63;
@@ -487,7 +474,7 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
                     if (p.mask_kind & FA_MASK_SLIDING_WINDOW) lo = max(lo, q - p.window + 1 - col0);
                 }
             }
-            const float* vl = nullptr;   // dK/dV kernel: the stage's lse and Delta of the columns
+            const float* vl = nullptr;   // dK/dV pass: the stage's lse and Delta of the columns
             const float* vd = nullptr;
             if constexpr (KV) {
                 const uint8_t* st = reinterpret_cast<const uint8_t*>(__cvta_shared_to_generic(
@@ -495,7 +482,6 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
                 vl = reinterpret_cast<const float*>(st) + 64 * g;
                 vd = reinterpret_cast<const float*>(st + 512) + 64 * g;
             }
-            uint32_t pk[2][16], dk[2][16];
             // Column c's bias is slope * (kv - q): +1 per column in the dQ pass (kv grows),
             // -1 per column in the dK/dV pass (q grows).  Pairs of columns in packed f32x2.
             const float bias0 = KV ? slope_log2 * (float)(row_pos - col0) : slope_log2 * (float)(col0 - row_pos);
@@ -507,13 +493,14 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
             const float2 cap2 = make_float2(p.softcap_log2, p.softcap_log2);
             const float2 nrl2 = make_float2(-row_l, -row_l), nrd2 = make_float2(-row_d, -row_d);
             const float2 one2 = make_float2(1.f, 1.f);
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
+            // P and dS of one 32-column half (h2) of this group's 64 columns, in 16-bit pairs.
+            auto half = [&](int h2, const uint32_t (&sr)[32], const uint32_t (&dr)[32], uint32_t (&pk)[16],
+                            uint32_t (&dk)[16]) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int c = 32 * h2 + 2 * i;
-                    const float2 raw = make_float2(__uint_as_float(sr[h2][2 * i]), __uint_as_float(sr[h2][2 * i + 1]));
-                    const float2 dp = make_float2(__uint_as_float(dr[h2][2 * i]), __uint_as_float(dr[h2][2 * i + 1]));
+                    const float2 raw = make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+                    const float2 dp = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
                     float2 x, th;
                     if constexpr (kSoftcap) {
                         const float2 a = __fmul2_rn(raw, inv2);
@@ -545,22 +532,58 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
                     }
                     float2 ds = __fmul2_rn(pr, __fadd2_rn(dp, nd));
                     if constexpr (kSoftcap) ds = __fmul2_rn(ds, __ffma2_rn(make_float2(-th.x, -th.y), th, one2));
-                    pk[h2][i] = pack2<BF16>(pr.x, pr.y);
-                    dk[h2][i] = pack2<BF16>(ds.x, ds.y);
+                    pk[i] = pack2<BF16>(pr.x, pr.y);
+                    dk[i] = pack2<BF16>(ds.x, ds.y);
                 }
-            }
+            };
+            uint32_t pk0[16], dk0[16];
             if constexpr (C::kSep) {
-                // The last entry's accumulating MMAs read the P / dS columns: wait for them.
+                // Half 0, then half 1's loads; once both halves of S and dP are in registers the
+                // MMA warp may compute the next entry's into them.  P and dS go to their own
+                // columns after the last entry's accumulating MMAs have read those.
+                {
+                    uint32_t sr[32], dr[32];
+                    tmem_ld_32x32b_x32(tS, sr);
+                    tmem_ld_32x32b_x32(tDP, dr);
+                    tmem_ld_wait();
+                    reg_fence<32>(sr);
+                    reg_fence<32>(dr);
+                    half(0, sr, dr, pk0, dk0);
+                }
+                uint32_t sr[32], dr[32], pk1[16], dk1[16];
+                tmem_ld_32x32b_x32(tS + 32, sr);
+                tmem_ld_32x32b_x32(tDP + 32, dr);
+                tmem_ld_wait();
+                reg_fence<32>(sr);
+                reg_fence<32>(dr);
+                tc_fence_before();
+                mbar_arrive_warp(bar(kBbLoaded));
+                half(1, sr, dr, pk1, dk1);
                 if (!wait(kBbAccDone, (ad_iter & 1u) ^ 1u)) { ok = false; break; }
                 ++ad_iter;
                 tc_fence_after();
+                if constexpr (KV) {
+                    tmem_st_32x32b_x16(tP, pk0);
+                    tmem_st_32x32b_x16(tP + 16, pk1);
+                }
+                tmem_st_32x32b_x16(tDS, dk0);
+                tmem_st_32x32b_x16(tDS + 16, dk1);
+            } else {
+                // Over the group's own columns, half by half: each half's P and dS land on S and
+                // dP columns this group has already read.
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t sr[32], dr[32];
+                    tmem_ld_32x32b_x32(tS + 32 * h2, sr);
+                    tmem_ld_32x32b_x32(tDP + 32 * h2, dr);
+                    tmem_ld_wait();
+                    reg_fence<32>(sr);
+                    reg_fence<32>(dr);
+                    half(h2, sr, dr, pk0, dk0);
+                    if constexpr (KV) tmem_st_32x32b_x16(tP + 16 * h2, pk0);
+                    tmem_st_32x32b_x16(tDS + 16 * h2, dk0);
+                }
             }
-            if constexpr (KV) {
-                tmem_st_32x32b_x16(tP, pk[0]);
-                tmem_st_32x32b_x16(tP + 16, pk[1]);
-            }
-            tmem_st_32x32b_x16(tDS, dk[0]);
-            tmem_st_32x32b_x16(tDS + 16, dk[1]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive_warp(bar(kBbPReady));
