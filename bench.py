@@ -105,28 +105,52 @@ def _strip_c_comments(text: str) -> str:
     return " ".join("".join(out).split())
 
 
-def kernel_source_sha() -> str:
-    """Hash of the forward kernel's code (comments and layout ignored), to tell whether the
+# The code of each kernel family: its own sources plus the parameter struct it is launched
+# with (extracted from the shared header), so edits elsewhere leave its recorded counters valid.
+KERNEL_SOURCES = {
+    "forward": (["block_sparse_masked_x128_b200/csrc/attn_fwd.cu",
+                 "block_sparse_masked_x128_b200/csrc/fwd_common.cuh",
+                 "block_sparse_masked_x128_b200/csrc/sm100_ptx.cuh"], "FwdParams"),
+    "backward": (["block_sparse_masked_x128_b200/csrc/attn_bwd.cu",
+                  "block_sparse_masked_x128_b200/csrc/fwd_common.cuh",
+                  "block_sparse_masked_x128_b200/csrc/sm100_ptx.cuh"], "BwdParams"),
+    "masked_softmax": (["block_sparse_masked_x128_b200/csrc/masked_softmax.cu",
+                        "block_sparse_masked_x128_b200/csrc/sm100_ptx.cuh"], None),
+    "decode": (["block_sparse_masked_x128_b200/csrc/decode.cu",
+                "block_sparse_masked_x128_b200/csrc/sm100_ptx.cuh"], "DecodeParams"),
+}
+
+
+def _struct_text(header_text: str, name: str) -> str:
+    i = header_text.find("struct %s {" % name)
+    if i < 0:
+        return ""
+    return header_text[i:header_text.find("};", i) + 2]
+
+
+def kernel_source_sha(family: str = "forward") -> str:
+    """Hash of one kernel family's code (comments and layout ignored), to tell whether the
     recorded ncu counters still describe the kernel that runs."""
+    files, struct = KERNEL_SOURCES[family]
     h = hashlib.sha256()
-    for rel in ("block_sparse_masked_x128_b200/csrc/attn_fwd.cu",
-                "block_sparse_masked_x128_b200/csrc/fwd_common.cuh",
-                "block_sparse_masked_x128_b200/csrc/sm100_ptx.cuh",
-                "block_sparse_masked_x128_b200/csrc/fa_internal.h", "include/fa_b200.h"):
+    for rel in files:
         with open(os.path.join(ROOT, rel), encoding="utf-8") as fh:
             h.update(_strip_c_comments(fh.read()).encode())
+    if struct:
+        with open(os.path.join(ROOT, "block_sparse_masked_x128_b200/csrc/fa_internal.h"), encoding="utf-8") as fh:
+            h.update(_strip_c_comments(_struct_text(fh.read(), struct)).encode())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(name: str, family: str = "forward"):
     """DRAM bytes per launch from the committed ncu summary, if taken on this kernel source."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(workload)
-    if not e or e.get("kernel_source_sha") != kernel_source_sha():
+    e = d.get(name)
+    if not e or e.get("kernel_source_sha") != kernel_source_sha(family):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -425,7 +449,8 @@ def time_masked_softmax(w: wl.SoftmaxWorkload, steps: int, warmup: int, world: i
                        "offset": w.offset, "dtype": w.dtype},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "traffic": None, "peak_source": peaks["source"] + " hbm_gbs",
+                         "traffic": recorded_traffic(w.name, "masked_softmax"),
+                         "peak_source": peaks["source"] + " hbm_gbs",
                          "kernel": "masked_softmax_kernel"},
             "clocks": clocks.summary()}
 
@@ -482,7 +507,8 @@ def time_backward(w: wl.Workload, steps: int, warmup: int, world: int, rank: int
             "executed_gflop_per_step": flops * 1.4 / 1e9, "gpu_launches": 3 * steps,
             "config": {"workload": w.name, "dtype": w.dtype},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": recorded_traffic("backward_" + w.name, "backward"),
                          "peak_source": peaks["source"] + " bf16_tflops (burst)",
                          "kernel": "attn_bwd_kernel (dK/dV and dQ passes) + pre-pass"},
             "clocks": clocks.summary()}
@@ -541,8 +567,10 @@ def time_decode(w: wl.DecodeWorkload, steps: int, warmup: int, world: int, dev) 
                        "context_lengths": f"seeded in [{w.lo}, {w.hi}]", "dtype": w.dtype,
                        "pages": int(sum(-(-int(n) // 128) for n in lens))},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                         "peak_source": peaks["source"] + " hbm_gbs", "kernel": "attn_fwd_kernel (paged)"},
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": recorded_traffic(w.name, "decode"),
+                         "peak_source": peaks["source"] + " hbm_gbs",
+                         "kernel": "decode_split_kernel + decode_merge_kernel"},
             "clocks": clocks.summary()}
 
 

@@ -537,10 +537,33 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
                 }
             };
             uint32_t pk0[16], dk0[16];
-            if constexpr (C::kSep) {
-                // Half 0, then half 1's loads; once both halves of S and dP are in registers the
-                // MMA warp may compute the next entry's into them.  P and dS go to their own
-                // columns after the last entry's accumulating MMAs have read those.
+            if constexpr (C::kSep && !KV) {
+                // dQ pass (dS only): both halves of S and dP into registers at once, so the MMA
+                // warp computes the next entry's S and dP during all of this entry's math (at
+                // D = 128 those MMAs take longer than the math).
+                uint32_t sr0[32], dr0[32], sr1[32], dr1[32], dk1[16];
+                tmem_ld_32x32b_x32(tS, sr0);
+                tmem_ld_32x32b_x32(tDP, dr0);
+                tmem_ld_32x32b_x32(tS + 32, sr1);
+                tmem_ld_32x32b_x32(tDP + 32, dr1);
+                tmem_ld_wait();
+                reg_fence<32>(sr0);
+                reg_fence<32>(dr0);
+                reg_fence<32>(sr1);
+                reg_fence<32>(dr1);
+                tc_fence_before();
+                mbar_arrive_warp(bar(kBbLoaded));
+                half(0, sr0, dr0, pk0, dk0);
+                half(1, sr1, dr1, pk0, dk1);
+                if (!wait(kBbAccDone, (ad_iter & 1u) ^ 1u)) { ok = false; break; }
+                ++ad_iter;
+                tc_fence_after();
+                tmem_st_32x32b_x16(tDS, dk0);
+                tmem_st_32x32b_x16(tDS + 16, dk1);
+            } else if constexpr (C::kSep) {
+                // dK/dV pass: half 0, then half 1's loads; once both halves of S and dP are in
+                // registers the MMA warp may compute the next entry's into them.  P and dS go to
+                // their own columns after the last entry's accumulating MMAs have read those.
                 {
                     uint32_t sr[32], dr[32];
                     tmem_ld_32x32b_x32(tS, sr);

@@ -62,9 +62,11 @@ __device__ __forceinline__ float dtype_min() {
     return BF16 ? -3.38953138925153547590e38f : -65504.0f;
 }
 
+// Two 16-bit values (lo in bits 0-15) as floats.
 template <bool BF16>
-__device__ __forceinline__ float to_f32(uint32_t bits16) {
-    return BF16 ? __uint_as_float(bits16 << 16) : __half2float(__ushort_as_half((unsigned short)bits16));
+__device__ __forceinline__ float2 to_f32x2(uint32_t w) {
+    if constexpr (BF16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
 
 __device__ __forceinline__ int64_t live_keys(const SoftmaxParams& p, int64_t q) {
@@ -219,30 +221,40 @@ __global__ void __launch_bounds__(kSmThreads, 1) masked_softmax_kernel(const __g
         const int64_t n_live = live_keys(p, q);
         const uint16_t* srow = reinterpret_cast<const uint16_t*>(smem + (size_t)s * p.stage_bytes);
 
-        // Pass 1: the selected values in registers, and the row max.
-        float x[VPT * 8];
-        float m = -INFINITY;
+        // Pass 1: the selected values in registers (pairs), and the row max.  32-bit indices
+        // (K <= 32768); vectors wholly inside the live prefix need no select.
+        const int K = p.K, nl = (int)n_live;
+        float2 x[VPT * 4];
+        float mc0 = -INFINITY, mc1 = -INFINITY;
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-            const int64_t e0 = 8ll * (c + kSmCompute * j);
-            if (e0 >= p.K) {
+            const int e0 = 8 * (c + kSmCompute * j);
+            if (e0 >= K) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) x[8 * j + i] = -INFINITY;   // past the row: no key
-            } else if (e0 >= n_live) {
+                for (int i = 0; i < 4; ++i) x[4 * j + i] = make_float2(-INFINITY, -INFINITY);   // no key
+            } else if (e0 >= nl) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) x[8 * j + i] = kMasked;
-                m = fmaxf(m, kMasked);
+                for (int i = 0; i < 4; ++i) x[4 * j + i] = make_float2(kMasked, kMasked);
+                mc0 = fmaxf(mc0, kMasked);
             } else {
                 const uint4 raw = *reinterpret_cast<const uint4*>(srow + e0);
                 const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float v = to_f32<BF16>((w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
-                    x[8 * j + i] = (e0 + i < n_live) ? v : kMasked;
-                    m = fmaxf(m, x[8 * j + i]);
+                for (int i = 0; i < 4; ++i) x[4 * j + i] = to_f32x2<BF16>(w[i]);
+                if (e0 + 8 > nl) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (e0 + 2 * i >= nl) x[4 * j + i].x = kMasked;
+                        if (e0 + 2 * i + 1 >= nl) x[4 * j + i].y = kMasked;
+                    }
                 }
+                mc0 = max3(mc0, x[4 * j].x, x[4 * j].y);
+                mc1 = max3(mc1, x[4 * j + 1].x, x[4 * j + 1].y);
+                mc0 = max3(mc0, x[4 * j + 2].x, x[4 * j + 2].y);
+                mc1 = max3(mc1, x[4 * j + 3].x, x[4 * j + 3].y);
             }
         }
+        float m = fmaxf(mc0, mc1);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
         if (lane == 0) red_max[cw] = m;
@@ -251,26 +263,30 @@ __global__ void __launch_bounds__(kSmThreads, 1) masked_softmax_kernel(const __g
 #pragma unroll
         for (int w = 1; w < kSmCompute / 32; ++w) m = fmaxf(m, red_max[w]);
 
-        // Pass 2: e = 2^((x - m) log2 e) and the row sum, in a fixed order.  A vector wholly
-        // past the causal boundary holds exp(finfo.min - m) = 0 unless the whole row is
-        // masked (m == finfo.min), where it is computed like any other.
-        float sum = 0.f;
+        // Pass 2: e = 2^((x - m) log2 e) and the row sum, in a fixed order (two running sums
+        // over the pairs' halves).  A vector wholly past the causal boundary holds
+        // exp(finfo.min - m) = 0 unless the whole row is masked (m == finfo.min), where it is
+        // computed like any other.
+        const float2 nm2 = make_float2(-m, -m), l2e = make_float2(kSmLog2e, kSmLog2e);
+        float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-            const int64_t e0 = 8ll * (c + kSmCompute * j);
-            if (e0 >= p.K) continue;
-            if (e0 >= n_live && m != kMasked) {
+            const int e0 = 8 * (c + kSmCompute * j);
+            if (e0 >= K) continue;
+            if (e0 >= nl && m != kMasked) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) x[8 * j + i] = 0.f;
+                for (int i = 0; i < 4; ++i) x[4 * j + i] = make_float2(0.f, 0.f);
                 continue;
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float e = ex2_approx((x[8 * j + i] - m) * kSmLog2e);
-                x[8 * j + i] = e;
-                sum += e;
+            for (int i = 0; i < 4; ++i) {
+                const float2 t = __fmul2_rn(__fadd2_rn(x[4 * j + i], nm2), l2e);
+                const float2 e = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                x[4 * j + i] = e;
+                sum2 = __fadd2_rn(sum2, e);
             }
         }
+        float sum = sum2.x + sum2.y;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o);
         if (lane == 0) red_sum[cw] = sum;
@@ -279,16 +295,20 @@ __global__ void __launch_bounds__(kSmThreads, 1) masked_softmax_kernel(const __g
 #pragma unroll
         for (int w = 1; w < kSmCompute / 32; ++w) sum += red_sum[w];
         const float inv = 1.0f / sum;
+        const float2 inv2 = make_float2(inv, inv);
 
         // Pass 3: p = e / sum as 16-bit values over the buffer; the producer stores it.
         uint16_t* wrow = reinterpret_cast<uint16_t*>(smem + (size_t)s * p.stage_bytes);
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-            const int64_t e0 = 8ll * (c + kSmCompute * j);
-            if (e0 >= p.K) continue;
+            const int e0 = 8 * (c + kSmCompute * j);
+            if (e0 >= K) continue;
             uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) w[i] = pack2<BF16>(x[8 * j + 2 * i] * inv, x[8 * j + 2 * i + 1] * inv);
+            for (int i = 0; i < 4; ++i) {
+                const float2 pr = __fmul2_rn(x[4 * j + i], inv2);
+                w[i] = pack2<BF16>(pr.x, pr.y);
+            }
             *reinterpret_cast<uint4*>(wrow + e0) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();

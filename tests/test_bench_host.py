@@ -116,7 +116,7 @@ def test_peaks_and_recorded_traffic(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.read_peaks()["source"] == "fallback"
     os.makedirs(tmp_path / "profiles")
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "abc")
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda family="forward": "abc")
     (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(
         {"w1": {"kernel_source_sha": "abc", "dram_bytes_per_launch": 123},
          "w2": {"kernel_source_sha": "old", "dram_bytes_per_launch": 456}}))
@@ -157,3 +157,8 @@ def test_kernel_hash_ignores_comments_and_layout():
     assert "not a comment" in bench._strip_c_comments(a)
     assert bench._strip_c_comments("int x = 1;") != bench._strip_c_comments("int x = 2;")
     assert len(bench.kernel_source_sha()) == 16
+    assert {len(bench.kernel_source_sha(f)) for f in bench.KERNEL_SOURCES} == {16}
+    assert len({bench.kernel_source_sha(f) for f in bench.KERNEL_SOURCES}) == len(bench.KERNEL_SOURCES)
+    # Only a kernel's own struct enters its hash: the forward's ignores BwdParams.
+    text = "struct FwdParams { int a; };\nstruct BwdParams { int b; };"
+    assert bench._struct_text(text, "BwdParams") == "struct BwdParams { int b; };"
