@@ -81,7 +81,10 @@ struct BCfg {
     static constexpr int kBarUEmpty = kBbUnitEmpty;
     static constexpr int kBarSlotFull = kBbSlot;
     static constexpr int kBarSlotEmpty = kBbSlot + kStages;
-    static constexpr int kNumBars = kBbSlot + 2 * kStages;
+    // Half-step barriers of the dK/dV pass at D = 128 (S / dP full, P / dS ready), per buffer.
+    static constexpr int kBarSFullH = kBbSlot + 2 * kStages;
+    static constexpr int kBarPReadyH = kBarSFullH + 2;
+    static constexpr int kNumBars = kBarPReadyH + 2;
     static constexpr int kStageOff = 2 * kTileBytes;
     static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;   // + alignment slack
@@ -93,6 +96,11 @@ struct BCfg {
     // first 32 columns of its own 64 S and dP columns (group g: 64g.., 128 + 64g..), and the
     // MMAs and the element-wise pass alternate.
     static constexpr bool kSep = KV ? (D == 64) : true;
+    // The dK/dV pass at D = 128 works in half-steps of 64 queries: S^T and dP^T of a half are
+    // 64 columns each, in two buffers (columns 0-127 and 128-255), so the MMAs of half k + 1 run
+    // while the math warps work on half k; the 16-bit P and dS of a half are written over the
+    // first 16 of each group's 32 S and dP columns in the half's buffer.
+    static constexpr bool kHalves = KV && D == 128;
     static constexpr uint32_t kAccEnd = KV ? 256 + 2 * D : 256 + D;
     static constexpr uint32_t kColP = kSep ? kAccEnd : kColS;
     static constexpr uint32_t kColDS = kSep ? (KV ? kAccEnd + 64 : kAccEnd) : kColDP;
@@ -639,6 +647,251 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
     }
 }
 
+// ------------------------------------------------------------------ dK/dV pass in half-steps (D = 128)
+
+template <int D, bool BF16>
+__device__ void bwd_mma_halves(const BwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                               const volatile int* ring, volatile int* abort_flag) {
+    using C = BCfg<D, true>;
+    const uint32_t leader = elect_one_lane();
+    constexpr uint32_t kIdescS = make_idesc_f16(BF16, 128, 64, false);   // N = 64 queries
+    constexpr uint32_t kIdescAcc = make_idesc_f16(BF16, 128, D, true);
+    auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+    auto wait = [&](int i, uint32_t par) {
+        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
+    };
+    // D[128 x 64] = A[128 x D] B[64 x D]^T: B is 64 rows of a 128-row stage tile (its start
+    // address moved by 64 rows = 8 KB, a whole number of 1 KB swizzle atoms).
+    auto issue_ss64 = [&](uint32_t dcol, uint32_t a, uint32_t b) {
+        const uint64_t ad = make_sdesc_sw128(a, 16, 1024);
+        const uint64_t bd = make_sdesc_sw128(b, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_ss_if(leader, tmem + dcol, ad + off, bd + off, kIdescS, kk > 0 ? 1u : 0u);
+        }
+    };
+    // D[128 x D] += A[128 x 64] B[64 x D]: A 16-bit pairs of the half (K step kk: group kk / 2,
+    // its columns 8 (kk % 2) ..), B 64 rows of a stage tile, MN-major.
+    auto issue_ts64 = [&](uint32_t dcol, uint32_t acol, uint32_t b, bool accumulate) {
+        const uint64_t bd = make_sdesc_sw128(b, 16384, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t aoff = (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8);
+            mma_ts_if(leader, tmem + dcol, tmem + acol + aoff, bd + (uint64_t)((kk * 2048) >> 4), kIdescAcc,
+                      (kk > 0 || accumulate) ? 1u : 0u);
+        }
+    };
+    auto stage0 = [&](uint32_t ps) { return sbase + C::kStageOff + (ps % C::kStages) * C::kStageBytes; };
+    uint32_t pos = 0, hs = 0, fix_iter = 0, acc_iter = 0, u_iter = 0;
+    uint32_t pr_iter[2] = {0u, 0u};
+    bool ok = true;
+    const uint32_t sFix0 = sbase, sFix1 = sbase + C::kTileBytes;
+    // S^T and dP^T of half-step k of the unit (entry pos0 + k / 2, queries 64 (k % 2) ..) into
+    // buffer (hs0 + k) % 2.
+    auto issue_half = [&](uint32_t pos0, uint32_t hs0, int k) -> bool {
+        const uint32_t ps = pos0 + (uint32_t)(k >> 1);
+        const int h = k & 1;
+        if (h == 0) {
+            if (!wait(C::kBarSlotFull + (int)(ps % C::kStages), (ps / C::kStages) & 1u)) return false;
+            tc_fence_after();
+        }
+        const uint32_t b = (hs0 + (uint32_t)k) & 1u;
+        const uint32_t st0 = stage0(ps) + 8192u * (uint32_t)h, st1 = st0 + C::kTileBytes;
+        issue_ss64(128u * b, sFix0, st0);         // S^T_h = K_j Q_h^T
+        issue_ss64(128u * b + 64u, sFix1, st1);   // dP^T_h = V_j dO_h^T
+        tc_commit_if(leader, bar(C::kBarSFullH + (int)b));
+        return true;
+    };
+    for (;;) {
+        const int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, ok);
+        if (u < 0) break;
+        const BUnit un = decode_bunit(p, u);
+        if (un.E == 0) continue;
+        if (!wait(kBbFixFull, fix_iter & 1u)) { ok = false; break; }
+        ++fix_iter;
+        tc_fence_after();
+        const uint32_t pos0 = pos, hs0 = hs;
+        const int K2 = 2 * un.E;
+        if (!issue_half(pos0, hs0, 0)) { ok = false; break; }
+        for (int k = 0; k < K2; ++k) {
+            // The next half's S^T and dP^T first: they overwrite the buffer of half k - 1, whose
+            // accumulating MMAs were issued before (one thread's MMAs run in issue order).
+            if (k + 1 < K2 && !issue_half(pos0, hs0, k + 1)) { ok = false; break; }
+            const uint32_t b = (hs0 + (uint32_t)k) & 1u;
+            if (!wait(C::kBarPReadyH + (int)b, pr_iter[b] & 1u)) { ok = false; break; }
+            ++pr_iter[b];
+            if (k == 0 && !wait(kBbAccFree, (acc_iter & 1u) ^ 1u)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t ps = pos0 + (uint32_t)(k >> 1);
+            const int h = k & 1;
+            const uint32_t st0 = stage0(ps) + 8192u * (uint32_t)h, st1 = st0 + C::kTileBytes;
+            issue_ts64(C::kColAcc0, 128u * b, st1, k > 0);         // dV += P^T_h dO_h
+            issue_ts64(C::kColAcc1, 128u * b + 64u, st0, k > 0);   // dK += dS^T_h Q_h
+            if (h == 1) tc_commit_if(leader, bar(C::kBarSlotEmpty + (int)(ps % C::kStages)));
+        }
+        if (!ok) break;
+        pos += (uint32_t)un.E;
+        hs += (uint32_t)K2;
+        tc_commit_if(leader, bar(kBbAccFull));
+        tc_commit_if(leader, bar(kBbFixEmpty));
+        ++acc_iter;
+    }
+    if (!ok) {
+        tc_commit_if(leader, bar(kBbDrain));
+        drain_wait(bar(kBbDrain), 0u);
+    }
+}
+
+template <int D, bool BF16, int VAR>
+__device__ void bwd_math_halves(const BwdParams& p, int g, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                                const volatile int* ring, volatile int* abort_flag) {
+    using C = BCfg<D, true>;
+    constexpr int SCORE = VAR & (FA_SCORE_SOFTCAP | FA_SCORE_ALIBI);
+    constexpr bool kDoc = (VAR & kVarDocumentB) != 0;
+    constexpr bool kSoftcap = (SCORE & FA_SCORE_SOFTCAP) != 0;
+    constexpr bool kAlibi = (SCORE & FA_SCORE_ALIBI) != 0;
+    const int wq = (threadIdx.x >> 5) & 3;
+    const int lane = threadIdx.x & 31;
+    const int r = wq * 32 + lane;                       // key row of the tile (TMEM lane)
+    const uint32_t lane_bits = (uint32_t)(wq * 32) << 16;
+    auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+    auto wait = [&](int i, uint32_t par) {
+        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
+    };
+    uint32_t pos = 0, hs = 0, acc_iter = 0, u_iter = 0;
+    uint32_t sf_iter[2] = {0u, 0u};
+    bool ok = true;
+    for (;;) {
+        const int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, ok);
+        if (u < 0) return;
+        const BUnit un = decode_bunit(p, u);
+        const int kv = un.idx * kBlock + r;
+        // Group 0 writes dV, group 1 dK (scaled).
+        const bool dk_row = (g == 1);
+        const int64_t* gst = dk_row ? p.grad0_stride : p.grad1_stride;
+        uint16_t* grow = reinterpret_cast<uint16_t*>(dk_row ? p.grad0 : p.grad1) + un.b * gst[0] +
+                         un.h * gst[1] + (int64_t)kv * gst[2];
+        const float gmul = dk_row ? p.scale : 1.0f;
+        const bool row_in = kv < p.KV_LEN;
+        if (un.E == 0) {
+            if (row_in) store_zero_cols(grow, D);
+            continue;
+        }
+        const float slope_log2 = kAlibi ? alibi_slope_log2(p, un.h) : 0.f;
+        const int row_doc = (kDoc && kv < p.QB * kBlock) ? __ldg(p.doc_id + kv) : 0;
+        const int kv_len = p.kv_lens ? min(p.KV_LEN, __ldg(p.kv_lens + (p.maskB == 1 ? 0 : un.b))) : p.KV_LEN;
+        EntryReader er;
+        er.init(un.entries, un.E);
+        for (int e = 0; e < un.E && ok; ++e) {
+            const int code = er.get(e);
+            int t = code & 0xFFFF;
+            FA_DCHECK_INDEX(t, p.entries_stride, p.status);
+            const bool full = (code & kFull0) != 0;
+            const int s = (int)(pos % C::kStages);
+            ++pos;
+            const uint8_t* stv = reinterpret_cast<const uint8_t*>(__cvta_shared_to_generic(
+                sbase + C::kStageOff + (uint32_t)s * C::kStageBytes + 2 * C::kTileBytes));
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t b = hs & 1u;
+                ++hs;
+                if (!wait(C::kBarSFullH + (int)b, sf_iter[b] & 1u)) { ok = false; break; }
+                ++sf_iter[b];
+                tc_fence_after();
+                const uint32_t tS = tmem + lane_bits + 128u * b + 32u * g;
+                const uint32_t tDP = tS + 64u;
+                uint32_t sr[32], dr[32];
+                tmem_ld_32x32b_x32(tS, sr);
+                tmem_ld_32x32b_x32(tDP, dr);
+                tmem_ld_wait();
+                reg_fence<32>(sr);
+                reg_fence<32>(dr);
+                // Columns: queries q = col0 + c, c in [0, 32).
+                const int col0 = t * kBlock + 64 * h + 32 * g;
+                int lo = 0, hi = 31;
+                if (!full) {
+                    if (kv >= kv_len) hi = -1;
+                    hi = min(hi, p.Q_LEN - 1 - col0);
+                    if (p.mask_kind & (FA_MASK_CAUSAL | FA_MASK_SLIDING_WINDOW)) lo = max(lo, kv - col0);
+                    if (p.mask_kind & FA_MASK_SLIDING_WINDOW) hi = min(hi, kv + p.window - 1 - col0);
+                }
+                const float* vl = reinterpret_cast<const float*>(stv) + 64 * h + 32 * g;
+                const float* vd = vl + kBlock;
+                float2 pos2 = make_float2(slope_log2 * (float)(kv - col0), slope_log2 * (float)(kv - col0 - 1));
+                const float2 step2 = make_float2(-2.f * slope_log2, -2.f * slope_log2);
+                const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+                const float2 inv2 = make_float2(p.inv_softcap_scale, p.inv_softcap_scale);
+                const float2 cap2 = make_float2(p.softcap_log2, p.softcap_log2);
+                const float2 one2 = make_float2(1.f, 1.f);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int c = 2 * i;
+                    const float2 raw = make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+                    const float2 dp = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
+                    float2 x, th;
+                    if constexpr (kSoftcap) {
+                        const float2 a = __fmul2_rn(raw, inv2);
+                        th = make_float2(tanh_approx(a.x), tanh_approx(a.y));
+                        x = __fmul2_rn(cap2, th);
+                    } else {
+                        x = __fmul2_rn(raw, sc2);
+                    }
+                    if constexpr (kAlibi) {
+                        x = __fadd2_rn(x, pos2);
+                        pos2 = __fadd2_rn(pos2, step2);
+                    }
+                    const float2 l2 = *reinterpret_cast<const float2*>(vl + c);
+                    const float2 d2 = *reinterpret_cast<const float2*>(vd + c);
+                    const float2 ex = __fadd2_rn(x, make_float2(-l2.x, -l2.y));
+                    float2 pr = make_float2(ex2_approx(ex.x), ex2_approx(ex.y));
+                    if (!full) {
+                        bool l0 = c >= lo && c <= hi, l1 = c + 1 >= lo && c + 1 <= hi;
+                        if constexpr (kDoc) {
+                            l0 = l0 && (__ldg(p.doc_id + col0 + c) == row_doc);
+                            l1 = l1 && (__ldg(p.doc_id + col0 + c + 1) == row_doc);
+                        }
+                        pr = make_float2(l0 ? pr.x : 0.f, l1 ? pr.y : 0.f);
+                    }
+                    float2 ds = __fmul2_rn(pr, __fadd2_rn(dp, make_float2(-d2.x, -d2.y)));
+                    if constexpr (kSoftcap) ds = __fmul2_rn(ds, __ffma2_rn(make_float2(-th.x, -th.y), th, one2));
+                    pk[i] = pack2<BF16>(pr.x, pr.y);
+                    dk[i] = pack2<BF16>(ds.x, ds.y);
+                }
+                // Over this group's own S and dP columns of the buffer, already read.
+                tmem_st_32x32b_x16(tS, pk);
+                tmem_st_32x32b_x16(tDP, dk);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive_warp(bar(C::kBarPReadyH + (int)b));
+            }
+        }
+        if (!ok) return;
+        if (!wait(kBbAccFull, acc_iter & 1u)) return;
+        ++acc_iter;
+        tc_fence_after();
+        const uint32_t tAcc = tmem + lane_bits + (dk_row ? C::kColAcc1 : C::kColAcc0);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(tAcc + 32 * c, o);
+            tmem_ld_wait();
+            reg_fence<32>(o);
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                w[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * gmul, __uint_as_float(o[2 * i + 1]) * gmul);
+            if (row_in) {
+                uint4* dst = reinterpret_cast<uint4*>(grow + 32 * c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+        }
+        tc_fence_before();
+        mbar_arrive_warp(bar(kBbAccFree));
+    }
+}
+
 // ------------------------------------------------------------------ kernels
 
 template <int D, bool BF16, int VAR, bool KV>
@@ -674,6 +927,10 @@ attn_bwd_kernel(const __grid_constant__ BwdParams p, const __grid_constant__ CUt
             mbar_init(bars + 8u * (C::kBarSlotFull + s), 1);
             mbar_init(bars + 8u * (C::kBarSlotEmpty + s), 1);
         }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bars + 8u * (C::kBarSFullH + b), 1);
+            mbar_init(bars + 8u * (C::kBarPReadyH + b), 8);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -690,11 +947,13 @@ attn_bwd_kernel(const __grid_constant__ BwdParams p, const __grid_constant__ CUt
         if (warp == 0) {
             bwd_producer<D, KV>(p, &tq, &tk, &tv, &tdo, sbase, bars, ring, abort_flag);
         } else if (warp == 1) {
-            bwd_mma<D, BF16, KV>(p, sbase, bars, tmem, ring, abort_flag);
+            if constexpr (C::kHalves) bwd_mma_halves<D, BF16>(p, sbase, bars, tmem, ring, abort_flag);
+            else bwd_mma<D, BF16, KV>(p, sbase, bars, tmem, ring, abort_flag);
         }
     } else {
         regs_inc<kRegsMathBwd>();
-        bwd_math<D, BF16, VAR, KV>(p, (warp - 4) >> 2, sbase, bars, tmem, ring, abort_flag);
+        if constexpr (C::kHalves) bwd_math_halves<D, BF16, VAR>(p, (warp - 4) >> 2, sbase, bars, tmem, ring, abort_flag);
+        else bwd_math<D, BF16, VAR, KV>(p, (warp - 4) >> 2, sbase, bars, tmem, ring, abort_flag);
     }
     tc_fence_before();
     __syncthreads();
