@@ -771,11 +771,11 @@ fa_status_t fa_backward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_ten
     const bool bf16 = q->dtype == FA_DTYPE_BF16;
     const int D = (int)q->D;
     const int q_pad = m->QB * fa::kBlock;
-    float* lse_log2 = static_cast<float*>(workspace);
-    float* delta = lse_log2 + (size_t)q->B * q->H * q_pad;
+    float* neg_lse_log2 = static_cast<float*>(workspace);
+    float* neg_delta = neg_lse_log2 + (size_t)q->B * q->H * q_pad;
 
     e = fa::launch_bwd_preprocess(out->data, out->stride, dout->data, dout->stride, lse, (int)q->B,
-                                  (int)q->H, (int)q->S, q_pad, D, bf16, lse_log2, delta, st);
+                                  (int)q->H, (int)q->S, q_pad, D, bf16, neg_lse_log2, neg_delta, st);
     if (e != cudaSuccess) return cuda_fail(e, "backward pre-pass launch");
 
     const float sc = (scale > 0.f) ? scale : (float)(1.0 / std::sqrt((double)q->D));
@@ -800,8 +800,8 @@ fa_status_t fa_backward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_ten
     p.softcap_log2 = cap * 1.4426950408889634f;
     p.inv_softcap_scale = sc / cap;
     p.alibi_slopes = params ? params->alibi_slopes : nullptr;
-    p.lse_log2 = lse_log2;
-    p.delta = delta;
+    p.neg_lse_log2 = neg_lse_log2;
+    p.neg_delta = neg_delta;
     p.q_pad = q_pad;
     p.status = m->status;
     p.stall_loads = g_stall_loads.load(std::memory_order_relaxed);

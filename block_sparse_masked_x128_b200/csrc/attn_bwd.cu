@@ -44,6 +44,13 @@
 #include "sm100_ptx.cuh"
 #include "fwd_common.cuh"
 
+#ifdef FA_TRACE
+// The backward's own trace buffer (the tracer's device pointer is per translation unit).
+extern "C" int fa_debug_set_trace_buffer_bwd(void* device_ptr) {
+    return (int)cudaMemcpyToSymbol(g_fa_trace, &device_ptr, sizeof(device_ptr));
+}
+#endif
+
 namespace fa {
 namespace {
 
@@ -186,6 +193,7 @@ __device__ void bwd_producer(const BwdParams& p, const CUtensorMap* tq, const CU
     };
     uint32_t pos = 0, fix_iter = 0, u_iter = 0;
     bool ok = true;
+    FA_TRACE_DECL
     for (;;) {
         int u = -1;
         if (leader) {
@@ -206,7 +214,9 @@ __device__ void bwd_producer(const BwdParams& p, const CUtensorMap* tq, const CU
         if (u < 0) break;
         const BUnit un = decode_bunit(p, u);
         if (un.E == 0) continue;
+        FA_TRACE_EV(KV ? 0 : 12, 32);
         if (!wait(kBbFixEmpty, (fix_iter & 1u) ^ 1u)) { ok = false; break; }
+        FA_TRACE_EV(KV ? 0 : 12, 33);
         mbar_arrive_expect_tx_if(leader, bar(kBbFixFull), (uint32_t)(2 * C::kTileBytes));
         for (int c = 0; c < C::kChunks; ++c) {
             tma_load_4d_if(leader, sbase + c * 16384, fix0, bar(kBbFixFull), c * 64, un.idx * kBlock,
@@ -227,7 +237,9 @@ __device__ void bwd_producer(const BwdParams& p, const CUtensorMap* tq, const CU
             int t = er.get(e) & 0xFFFF;
             FA_DCHECK_INDEX(t, p.entries_stride, p.status);
             const int s = (int)(pos % C::kStages);
+            FA_TRACE_EV(KV ? 0 : 12, 30);
             if (!wait(C::kBarSlotEmpty + s, ((pos / C::kStages) & 1u) ^ 1u)) { ok = false; break; }
+            FA_TRACE_EV(KV ? 0 : 12, 31);
             const uint32_t dst = sbase + C::kStageOff + (uint32_t)s * C::kStageBytes;
             mbar_arrive_expect_tx_if(leader, bar(C::kBarSlotFull + s),
                                      (uint32_t)(2 * C::kTileBytes + C::kVecBytes));
@@ -239,9 +251,9 @@ __device__ void bwd_producer(const BwdParams& p, const CUtensorMap* tq, const CU
             }
             if constexpr (KV) {
                 if (leader) {
-                    bulk_load(dst + 2 * C::kTileBytes, p.lse_log2 + vec_row + (size_t)t * kBlock, 512,
+                    bulk_load(dst + 2 * C::kTileBytes, p.neg_lse_log2 + vec_row + (size_t)t * kBlock, 512,
                               bar(C::kBarSlotFull + s));
-                    bulk_load(dst + 2 * C::kTileBytes + 512, p.delta + vec_row + (size_t)t * kBlock, 512,
+                    bulk_load(dst + 2 * C::kTileBytes + 512, p.neg_delta + vec_row + (size_t)t * kBlock, 512,
                               bar(C::kBarSlotFull + s));
                 }
                 __syncwarp();
@@ -299,6 +311,7 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
     uint32_t pos = 0, fix_iter = 0, acc_iter = 0, pr_iter = 0, ld_iter = 0, u_iter = 0;
     bool ok = true;
     const uint32_t sFix0 = sbase, sFix1 = sbase + C::kTileBytes;
+    FA_TRACE_DECL
     auto stage0 = [&](uint32_t ps) { return sbase + C::kStageOff + (ps % C::kStages) * C::kStageBytes; };
     // S (or S^T) and dP (or dP^T) of the entry at ring position ps.
     auto issue_s_dp = [&](uint32_t ps) -> bool {
@@ -316,7 +329,9 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
         if (u < 0) break;
         const BUnit un = decode_bunit(p, u);
         if (un.E == 0) continue;
+        FA_TRACE_EV(KV ? 1 : 13, 20);
         if (!wait(kBbFixFull, fix_iter & 1u)) { ok = false; break; }
+        FA_TRACE_EV(KV ? 1 : 13, 21);
         ++fix_iter;
         tc_fence_after();
         if constexpr (C::kSep) {
@@ -327,7 +342,9 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
             if constexpr (C::kSep) {
                 // The next entry's S and dP as soon as the math warps hold this entry's.
                 if (e + 1 < un.E) {
+                    FA_TRACE_EV(KV ? 1 : 13, 22);
                     if (!wait(kBbLoaded, ld_iter & 1u)) { ok = false; break; }
+                    FA_TRACE_EV(KV ? 1 : 13, 23);
                     ++ld_iter;
                     if (!issue_s_dp(ps + 1)) { ok = false; break; }
                 } else {
@@ -337,7 +354,9 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
             } else {
                 if (!issue_s_dp(ps)) { ok = false; break; }
             }
+            FA_TRACE_EV(KV ? 1 : 13, 24);
             if (!wait(kBbPReady, pr_iter & 1u)) { ok = false; break; }
+            FA_TRACE_EV(KV ? 1 : 13, 25);
             ++pr_iter;
             if (e == 0 && !wait(kBbAccFree, (acc_iter & 1u) ^ 1u)) { ok = false; break; }
             tc_fence_after();
@@ -387,6 +406,57 @@ __device__ __forceinline__ void store_zero_cols(uint16_t* row, int cols) {
     for (int d = 0; d < cols; d += 8) *reinterpret_cast<uint4*>(row + d) = make_uint4(0, 0, 0, 0);
 }
 
+// Per-row constants of the element-wise pass.
+struct PairConsts {
+    float2 sc2, inv2, cap2, step2;
+    int lo, hi;             // live columns [lo, hi] of the row on a partial tile
+    int row_doc;
+    const int* doc_cols;    // document id of column 0 of the 32 (partial tiles with documents)
+};
+
+// P and dS of 32 columns of one row (16 pairs) from S and dP read out of TMEM, as 16-bit pairs:
+//   x = score_mod(s) in log2 units,  P = 2^(x + nl),  dS = P (dP + nd) (1 - tanh^2 under a cap),
+// with nl = -lse log2(e) and nd = -Delta of the pair's columns (nlv(i) / ndv(i)).  PART: the
+// tile is partial, so columns outside [lo, hi] (and of another document) get P = 0.
+template <bool BF16, int SCORE, bool DOC, bool PART, typename NL, typename ND>
+__device__ __forceinline__ void bwd_pairs(const uint32_t (&sr)[32], const uint32_t (&dr)[32],
+                                          const PairConsts& k, float2& pos2, NL nlv, ND ndv,
+                                          uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+    constexpr bool kSoftcap = (SCORE & FA_SCORE_SOFTCAP) != 0;
+    constexpr bool kAlibi = (SCORE & FA_SCORE_ALIBI) != 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int c = 2 * i;
+        const float2 raw = make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+        const float2 dp = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
+        const float2 nl = nlv(i);
+        float2 ex, th;
+        if constexpr (kSoftcap) {
+            const float2 a = __fmul2_rn(raw, k.inv2);
+            th = make_float2(tanh_approx(a.x), tanh_approx(a.y));
+            if constexpr (kAlibi) ex = __fadd2_rn(__ffma2_rn(k.cap2, th, pos2), nl);
+            else ex = __ffma2_rn(k.cap2, th, nl);
+        } else {
+            if constexpr (kAlibi) ex = __fadd2_rn(__ffma2_rn(raw, k.sc2, pos2), nl);
+            else ex = __ffma2_rn(raw, k.sc2, nl);
+        }
+        if constexpr (kAlibi) pos2 = __fadd2_rn(pos2, k.step2);
+        float2 pr = make_float2(ex2_approx(ex.x), ex2_approx(ex.y));
+        if constexpr (PART) {
+            bool l0 = c >= k.lo && c <= k.hi, l1 = c + 1 >= k.lo && c + 1 <= k.hi;
+            if constexpr (DOC) {
+                l0 = l0 && (__ldg(k.doc_cols + c) == k.row_doc);
+                l1 = l1 && (__ldg(k.doc_cols + c + 1) == k.row_doc);
+            }
+            pr = make_float2(l0 ? pr.x : 0.f, l1 ? pr.y : 0.f);
+        }
+        float2 ds = __fmul2_rn(pr, __fadd2_rn(dp, ndv(i)));
+        if constexpr (kSoftcap) ds = __fmul2_rn(ds, __ffma2_rn(make_float2(-th.x, -th.y), th, make_float2(1.f, 1.f)));
+        pk[i] = pack2<BF16>(pr.x, pr.y);
+        dk[i] = pack2<BF16>(ds.x, ds.y);
+    }
+}
+
 template <int D, bool BF16, int VAR, bool KV>
 __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          const volatile int* ring, volatile int* abort_flag) {
@@ -411,6 +481,8 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
     };
     uint32_t pos = 0, sf_iter = 0, acc_iter = 0, u_iter = 0, ld_iter = 0, ad_iter = 0;
     bool ok = true;
+    FA_TRACE_DECL
+    const int tslot = (threadIdx.x >> 5) + (KV ? 0 : 12);   // trace slot: warp, by pass
     for (;;) {
         const int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, ok);
         if (u < 0) return;
@@ -445,8 +517,8 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
         // dQ kernel: this thread's query row has one lse and one Delta.
         float row_l = 0.f, row_d = 0.f;
         if constexpr (!KV) {
-            row_l = __ldg(p.lse_log2 + vec_row + row_pos);
-            row_d = __ldg(p.delta + vec_row + row_pos);
+            row_l = __ldg(p.neg_lse_log2 + vec_row + row_pos);
+            row_d = __ldg(p.neg_delta + vec_row + row_pos);
         }
         const int row_doc = (kDoc && row_pos < p.QB * kBlock) ? __ldg(p.doc_id + row_pos) : 0;
         const int kv_len = p.kv_lens ? min(p.KV_LEN, __ldg(p.kv_lens + (p.maskB == 1 ? 0 : un.b))) : p.KV_LEN;
@@ -459,7 +531,9 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
             const bool full = (code & kFull0) != 0;
             const int s = (int)(pos % C::kStages);
             ++pos;
+            FA_TRACE_EV(tslot, 2);
             if (!wait(kBbSFull, sf_iter & 1u)) { ok = false; break; }
+            FA_TRACE_EV(tslot, 3);
             ++sf_iter;
             tc_fence_after();
             const int col0 = t * kBlock + 64 * g;        // first column position (q or kv)
@@ -495,54 +569,30 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
             const float bias0 = KV ? slope_log2 * (float)(row_pos - col0) : slope_log2 * (float)(col0 - row_pos);
             const float dbias = KV ? -slope_log2 : slope_log2;
             float2 pos2 = make_float2(bias0, bias0 + dbias);
-            const float2 step2 = make_float2(2.f * dbias, 2.f * dbias);
-            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-            const float2 inv2 = make_float2(p.inv_softcap_scale, p.inv_softcap_scale);
-            const float2 cap2 = make_float2(p.softcap_log2, p.softcap_log2);
-            const float2 nrl2 = make_float2(-row_l, -row_l), nrd2 = make_float2(-row_d, -row_d);
-            const float2 one2 = make_float2(1.f, 1.f);
+            PairConsts pc;
+            pc.sc2 = make_float2(p.scale_log2, p.scale_log2);
+            pc.inv2 = make_float2(p.inv_softcap_scale, p.inv_softcap_scale);
+            pc.cap2 = make_float2(p.softcap_log2, p.softcap_log2);
+            pc.step2 = make_float2(2.f * dbias, 2.f * dbias);
+            pc.row_doc = row_doc;
+            const float2 nrl2 = make_float2(row_l, row_l), nrd2 = make_float2(row_d, row_d);
             // P and dS of one 32-column half (h2) of this group's 64 columns, in 16-bit pairs.
             auto half = [&](int h2, const uint32_t (&sr)[32], const uint32_t (&dr)[32], uint32_t (&pk)[16],
                             uint32_t (&dk)[16]) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int c = 32 * h2 + 2 * i;
-                    const float2 raw = make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
-                    const float2 dp = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
-                    float2 x, th;
-                    if constexpr (kSoftcap) {
-                        const float2 a = __fmul2_rn(raw, inv2);
-                        th = make_float2(tanh_approx(a.x), tanh_approx(a.y));
-                        x = __fmul2_rn(cap2, th);
-                    } else {
-                        x = __fmul2_rn(raw, sc2);
-                    }
-                    if constexpr (kAlibi) {
-                        x = __fadd2_rn(x, pos2);
-                        pos2 = __fadd2_rn(pos2, step2);
-                    }
-                    float2 nl = nrl2, nd = nrd2;
-                    if constexpr (KV) {
-                        const float2 l2 = *reinterpret_cast<const float2*>(vl + c);
-                        const float2 d2 = *reinterpret_cast<const float2*>(vd + c);
-                        nl = make_float2(-l2.x, -l2.y);
-                        nd = make_float2(-d2.x, -d2.y);
-                    }
-                    const float2 ex = __fadd2_rn(x, nl);
-                    float2 pr = make_float2(ex2_approx(ex.x), ex2_approx(ex.y));
-                    if (!full) {
-                        bool l0 = c >= lo && c <= hi, l1 = c + 1 >= lo && c + 1 <= hi;
-                        if constexpr (kDoc) {
-                            l0 = l0 && (__ldg(p.doc_id + col0 + c) == row_doc);
-                            l1 = l1 && (__ldg(p.doc_id + col0 + c + 1) == row_doc);
-                        }
-                        pr = make_float2(l0 ? pr.x : 0.f, l1 ? pr.y : 0.f);
-                    }
-                    float2 ds = __fmul2_rn(pr, __fadd2_rn(dp, nd));
-                    if constexpr (kSoftcap) ds = __fmul2_rn(ds, __ffma2_rn(make_float2(-th.x, -th.y), th, one2));
-                    pk[i] = pack2<BF16>(pr.x, pr.y);
-                    dk[i] = pack2<BF16>(ds.x, ds.y);
-                }
+                PairConsts k = pc;
+                k.lo = lo - 32 * h2;
+                k.hi = hi - 32 * h2;
+                k.doc_cols = kDoc ? p.doc_id + col0 + 32 * h2 : nullptr;
+                auto nl = [&](int i) -> float2 {
+                    if constexpr (KV) return *reinterpret_cast<const float2*>(vl + 32 * h2 + 2 * i);
+                    else return nrl2;
+                };
+                auto nd = [&](int i) -> float2 {
+                    if constexpr (KV) return *reinterpret_cast<const float2*>(vd + 32 * h2 + 2 * i);
+                    else return nrd2;
+                };
+                if (full) bwd_pairs<BF16, SCORE, kDoc, false>(sr, dr, k, pos2, nl, nd, pk, dk);
+                else bwd_pairs<BF16, SCORE, kDoc, true>(sr, dr, k, pos2, nl, nd, pk, dk);
             };
             uint32_t pk0[16], dk0[16];
             if constexpr (C::kSep && !KV) {
@@ -561,9 +611,12 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
                 reg_fence<32>(dr1);
                 tc_fence_before();
                 mbar_arrive_warp(bar(kBbLoaded));
+                FA_TRACE_EV(tslot, 4);
                 half(0, sr0, dr0, pk0, dk0);
                 half(1, sr1, dr1, pk0, dk1);
+                FA_TRACE_EV(tslot, 5);
                 if (!wait(kBbAccDone, (ad_iter & 1u) ^ 1u)) { ok = false; break; }
+                FA_TRACE_EV(tslot, 6);
                 ++ad_iter;
                 tc_fence_after();
                 tmem_st_32x32b_x16(tDS, dk0);
@@ -589,8 +642,11 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
                 reg_fence<32>(dr);
                 tc_fence_before();
                 mbar_arrive_warp(bar(kBbLoaded));
+                FA_TRACE_EV(tslot, 4);
                 half(1, sr, dr, pk1, dk1);
+                FA_TRACE_EV(tslot, 5);
                 if (!wait(kBbAccDone, (ad_iter & 1u) ^ 1u)) { ok = false; break; }
+                FA_TRACE_EV(tslot, 6);
                 ++ad_iter;
                 tc_fence_after();
                 if constexpr (KV) {
@@ -618,10 +674,13 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive_warp(bar(kBbPReady));
+            FA_TRACE_EV(tslot, 7);
         }
         if (!ok) return;
         // Epilogue: this group's accumulator columns of the row, scaled, in the input dtype.
+        FA_TRACE_EV(tslot, 8);
         if (!wait(kBbAccFull, acc_iter & 1u)) return;
+        FA_TRACE_EV(tslot, 9);
         ++acc_iter;
         tc_fence_after();
         const uint32_t tAcc = tmem + lane_bits + (KV ? (g ? C::kColAcc1 : C::kColAcc0)
@@ -644,6 +703,7 @@ __device__ void bwd_math(const BwdParams& p, int g, uint32_t sbase, uint32_t bar
         }
         tc_fence_before();
         mbar_arrive_warp(bar(kBbAccFree));
+        FA_TRACE_EV(tslot, 10);
     }
 }
 
@@ -818,46 +878,20 @@ __device__ void bwd_math_halves(const BwdParams& p, int g, uint32_t sbase, uint3
                 const float* vl = reinterpret_cast<const float*>(stv) + 64 * h + 32 * g;
                 const float* vd = vl + kBlock;
                 float2 pos2 = make_float2(slope_log2 * (float)(kv - col0), slope_log2 * (float)(kv - col0 - 1));
-                const float2 step2 = make_float2(-2.f * slope_log2, -2.f * slope_log2);
-                const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-                const float2 inv2 = make_float2(p.inv_softcap_scale, p.inv_softcap_scale);
-                const float2 cap2 = make_float2(p.softcap_log2, p.softcap_log2);
-                const float2 one2 = make_float2(1.f, 1.f);
+                PairConsts k;
+                k.sc2 = make_float2(p.scale_log2, p.scale_log2);
+                k.inv2 = make_float2(p.inv_softcap_scale, p.inv_softcap_scale);
+                k.cap2 = make_float2(p.softcap_log2, p.softcap_log2);
+                k.step2 = make_float2(-2.f * slope_log2, -2.f * slope_log2);
+                k.lo = lo;
+                k.hi = hi;
+                k.row_doc = row_doc;
+                k.doc_cols = kDoc ? p.doc_id + col0 : nullptr;
+                auto nl = [&](int i) { return *reinterpret_cast<const float2*>(vl + 2 * i); };
+                auto nd = [&](int i) { return *reinterpret_cast<const float2*>(vd + 2 * i); };
                 uint32_t pk[16], dk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int c = 2 * i;
-                    const float2 raw = make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
-                    const float2 dp = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
-                    float2 x, th;
-                    if constexpr (kSoftcap) {
-                        const float2 a = __fmul2_rn(raw, inv2);
-                        th = make_float2(tanh_approx(a.x), tanh_approx(a.y));
-                        x = __fmul2_rn(cap2, th);
-                    } else {
-                        x = __fmul2_rn(raw, sc2);
-                    }
-                    if constexpr (kAlibi) {
-                        x = __fadd2_rn(x, pos2);
-                        pos2 = __fadd2_rn(pos2, step2);
-                    }
-                    const float2 l2 = *reinterpret_cast<const float2*>(vl + c);
-                    const float2 d2 = *reinterpret_cast<const float2*>(vd + c);
-                    const float2 ex = __fadd2_rn(x, make_float2(-l2.x, -l2.y));
-                    float2 pr = make_float2(ex2_approx(ex.x), ex2_approx(ex.y));
-                    if (!full) {
-                        bool l0 = c >= lo && c <= hi, l1 = c + 1 >= lo && c + 1 <= hi;
-                        if constexpr (kDoc) {
-                            l0 = l0 && (__ldg(p.doc_id + col0 + c) == row_doc);
-                            l1 = l1 && (__ldg(p.doc_id + col0 + c + 1) == row_doc);
-                        }
-                        pr = make_float2(l0 ? pr.x : 0.f, l1 ? pr.y : 0.f);
-                    }
-                    float2 ds = __fmul2_rn(pr, __fadd2_rn(dp, make_float2(-d2.x, -d2.y)));
-                    if constexpr (kSoftcap) ds = __fmul2_rn(ds, __ffma2_rn(make_float2(-th.x, -th.y), th, one2));
-                    pk[i] = pack2<BF16>(pr.x, pr.y);
-                    dk[i] = pack2<BF16>(ds.x, ds.y);
-                }
+                if (full) bwd_pairs<BF16, SCORE, kDoc, false>(sr, dr, k, pos2, nl, nd, pk, dk);
+                else bwd_pairs<BF16, SCORE, kDoc, true>(sr, dr, k, pos2, nl, nd, pk, dk);
                 // Over this group's own S and dP columns of the buffer, already read.
                 tmem_st_32x32b_x16(tS, pk);
                 tmem_st_32x32b_x16(tDP, dk);
@@ -999,8 +1033,8 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
     const uint16_t* __restrict__ out, int64_t os0, int64_t os1, int64_t os2,
     const uint16_t* __restrict__ dout, int64_t ds0, int64_t ds1, int64_t ds2,
-    const float* __restrict__ lse, int B, int H, int Q_LEN, int q_pad, float* __restrict__ lse_log2,
-    float* __restrict__ delta) {
+    const float* __restrict__ lse, int B, int H, int Q_LEN, int q_pad, float* __restrict__ neg_lse_log2,
+    float* __restrict__ neg_delta) {
     constexpr int kLanesPerRow = D / 8;          // one 16-byte vector per lane
     constexpr int kRowsPerWarp = 32 / kLanesPerRow;
     const int lane = threadIdx.x & 31;
@@ -1039,9 +1073,11 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
 #pragma unroll
     for (int o = kLanesPerRow / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(kFullMask, acc, o);
     if (row < total && sub == 0) {
-        delta[row] = (q < Q_LEN) ? acc : 0.f;
+        // Stored negated, so the main kernels add them (P = 2^(x + neg_lse_log2) and
+        // dP + neg_delta) with no negation per element.
+        neg_delta[row] = (q < Q_LEN) ? -acc : 0.f;
         const float l = (q < Q_LEN) ? lse[bh * Q_LEN + q] : -INFINITY;
-        lse_log2[row] = (l == -INFINITY) ? INFINITY : l * kLog2e;
+        neg_lse_log2[row] = (l == -INFINITY) ? -INFINITY : -(l * kLog2e);
     }
 }
 
@@ -1049,8 +1085,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
 
 cudaError_t launch_bwd_preprocess(const void* out, const int64_t out_stride[3], const void* dout,
                                   const int64_t dout_stride[3], const float* lse, int B, int H,
-                                  int Q_LEN, int q_pad, int D, bool bf16, float* lse_log2,
-                                  float* delta, cudaStream_t stream) {
+                                  int Q_LEN, int q_pad, int D, bool bf16, float* neg_lse_log2,
+                                  float* neg_delta, cudaStream_t stream) {
     const int64_t rows = (int64_t)B * H * q_pad;
     const int rows_per_warp = 32 / (D / 8);
     const int64_t warps = (rows + rows_per_warp - 1) / rows_per_warp;
@@ -1062,7 +1098,7 @@ cudaError_t launch_bwd_preprocess(const void* out, const int64_t out_stride[3], 
     if (D == DD && bf16 == BB) {                                                                    \
         bwd_preprocess_kernel<DD, BB><<<(unsigned)blocks, 256, 0, stream>>>(                        \
             o, out_stride[0], out_stride[1], out_stride[2], d, dout_stride[0], dout_stride[1],      \
-            dout_stride[2], lse, B, H, Q_LEN, q_pad, lse_log2, delta);                              \
+            dout_stride[2], lse, B, H, Q_LEN, q_pad, neg_lse_log2, neg_delta);                              \
         return cudaGetLastError();                                                                  \
     }
     FA_PRE(64, true)

@@ -131,8 +131,8 @@ struct BwdParams {
     float softcap_log2;           // softcap * log2(e)
     float inv_softcap_scale;      // scale / softcap
     const float* alibi_slopes;    // device [H] or null (then 2^(-8(h+1)/H))
-    const float* lse_log2;        // workspace [B*H][q_pad]: lse * log2(e), +inf without keys
-    const float* delta;           // workspace [B*H][q_pad]: rowsum(dO * O)
+    const float* neg_lse_log2;    // workspace [B*H][q_pad]: -lse * log2(e), -inf without keys
+    const float* neg_delta;       // workspace [B*H][q_pad]: -rowsum(dO * O)
     int32_t q_pad;                // QB * 128
     void* grad0;                  // dK/dV kernel: dK; dQ kernel: dQ
     void* grad1;                  // dK/dV kernel: dV; dQ kernel: unused
@@ -172,8 +172,8 @@ cudaError_t launch_decode(const DecodeParams& p, int D, bool bf16, int score_kin
 
 cudaError_t launch_bwd_preprocess(const void* out, const int64_t out_stride[3], const void* dout,
                                   const int64_t dout_stride[3], const float* lse, int B, int H,
-                                  int Q_LEN, int q_pad, int D, bool bf16, float* lse_log2,
-                                  float* delta, cudaStream_t stream);
+                                  int Q_LEN, int q_pad, int D, bool bf16, float* neg_lse_log2,
+                                  float* neg_delta, cudaStream_t stream);
 cudaError_t launch_attn_bwd_dkdv(const BwdParams& p, int D, bool bf16, int score_kind,
                                  const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                  const CUtensorMap& tdo, int grid, cudaStream_t stream);

@@ -1,4 +1,4 @@
-// fa_trace.cuh -- optional phase tracer of the forward kernel (compile-time FA_TRACE).
+// fa_trace.cuh -- optional phase tracer of the forward and backward kernels (compile-time FA_TRACE).
 //
 // Off by default: without FA_TRACE every trace point compiles to nothing.  The trace build
 // (build.py --trace, libfa_b200_trace.so) records, for CTA 0 only, a 64-bit word per
@@ -9,12 +9,13 @@
 #include <cstdint>
 
 namespace fa {
-constexpr int kTraceSlots = 20;
+constexpr int kTraceSlots = 24;
 constexpr int kTraceCap = 16384;
 }  // namespace fa
 
 #ifdef FA_TRACE
-// Defined in the one translation unit that includes this header (attn_fwd.cu).
+// One per translation unit that includes this header (attn_fwd.cu, attn_bwd.cu), each with
+// its own setter.
 static __device__ unsigned long long* g_fa_trace = nullptr;
 // Declares the role's trace cursor; the buffer pointer is read once, kept in a register.
 #define FA_TRACE_DECL                                                                \
