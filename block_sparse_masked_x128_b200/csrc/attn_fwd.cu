@@ -256,31 +256,30 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
 // P = 2^(x - base) for one 128-wide row, packed to 16-bit pairs and stored to TMEM at tP
 // in four 32-column chunks; returns the (two-lane) row sum.  EMU of every 16 pairs use
 // the FMA-pipe exp2 (only for tiles without masked positions), the rest MUFU ex2.
+// A warp issues in program order, so all 128 exponentials come first (overwriting x) and the
+// sums, packing and TMEM stores after them: the MUFU unit then gets one instruction per
+// issue opportunity instead of waiting at every chunk for the previous chunk's dependent work.
 template <bool BF16, bool SCORE, int EMU>
-__device__ __forceinline__ float2 softmax_p_row(const float2 (&x)[64], float2 nb2, float2 k2,
-                                                uint32_t tP) {
+__device__ __forceinline__ float2 softmax_p_row(float2 (&x)[64], float2 nb2, float2 k2, uint32_t tP) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const float2 a = SCORE ? __fadd2_rn(x[i], nb2) : __ffma2_rn(x[i], k2, nb2);
+        if (((i & 15) * EMU) % 16 < EMU) {
+            x[i] = exp2_fma2(a);
+        } else {
+            x[i] = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+        }
+    }
     float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                     make_float2(0.f, 0.f)};
 #pragma unroll
     for (int chunk = 0; chunk < 4; ++chunk) {
-        // All exponentials of the chunk first (independent, so their latencies overlap),
-        // then the sums and the 16-bit packing.
-        float2 pe[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float2 a = SCORE ? __fadd2_rn(x[chunk * 16 + i], nb2)
-                                   : __ffma2_rn(x[chunk * 16 + i], k2, nb2);
-            if ((i * EMU) % 16 < EMU) {
-                pe[i] = exp2_fma2(a);
-            } else {
-                pe[i] = make_float2(ex2_approx(a.x), ex2_approx(a.y));
-            }
-        }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            rs[i & 3] = __fadd2_rn(rs[i & 3], pe[i]);
-            pk[i] = pack2<BF16>(pe[i].x, pe[i].y);
+            const float2 pe = x[chunk * 16 + i];
+            rs[i & 3] = __fadd2_rn(rs[i & 3], pe);
+            pk[i] = pack2<BF16>(pe.x, pe.y);
         }
         tmem_st_32x32b_x16(tP + chunk * 16, pk);
     }
