@@ -108,10 +108,16 @@ struct BCfg {
     // while the math warps work on half k; the 16-bit P and dS of a half are written over the
     // first 16 of each group's 32 S and dP columns in the half's buffer.
     static constexpr bool kHalves = KV && D == 128;
+    // The dQ pass at D = 64 keeps its fixed tiles (Q_i, dO_i: the A operands of S and dP) in
+    // TMEM, copied there once per unit, so those MMAs read only B (K_j, V_j) from shared memory
+    // and the fixed tiles' shared memory is free for the next unit as soon as the copy is done.
+    static constexpr bool kTmemA = !KV && D == 64;
+    static constexpr uint32_t kColA0 = 384, kColA1 = 384 + D / 2;
     static constexpr uint32_t kAccEnd = KV ? 256 + 2 * D : 256 + D;
     static constexpr uint32_t kColP = kSep ? kAccEnd : kColS;
     static constexpr uint32_t kColDS = kSep ? (KV ? kAccEnd + 64 : kAccEnd) : kColDP;
     static_assert(!kSep || kColDS + 64 <= 512, "TMEM budget");
+    static_assert(!kTmemA || (kColA0 >= kColDS + 64 && kColA1 + D / 2 <= 512), "TMEM budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -308,6 +314,15 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
                       kIdescAcc, (kk > 0 || accumulate) ? 1u : 0u);
         }
     };
+    // D[128 x 128] = A B^T with A (128 x D, 16-bit pairs) in TMEM at acol, B K-major in smem.
+    auto issue_ts_a = [&](uint32_t dcol, uint32_t acol, uint32_t b) {
+        const uint64_t bd = make_sdesc_sw128(b, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_ts_if(leader, tmem + dcol, tmem + acol + 8u * (uint32_t)kk, bd + off, kIdescSS, kk > 0 ? 1u : 0u);
+        }
+    };
     uint32_t pos = 0, fix_iter = 0, acc_iter = 0, pr_iter = 0, ld_iter = 0, u_iter = 0;
     bool ok = true;
     const uint32_t sFix0 = sbase, sFix1 = sbase + C::kTileBytes;
@@ -319,8 +334,13 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
         if (!wait(C::kBarSlotFull + s, (ps / C::kStages) & 1u)) return false;
         tc_fence_after();
         const uint32_t st0 = stage0(ps), st1 = st0 + C::kTileBytes;
-        issue_ss(C::kColS, sFix0, st0);    // dK/dV pass: S^T = K_j Q_i^T;  dQ pass: S = Q_i K_j^T
-        issue_ss(C::kColDP, sFix1, st1);   // dK/dV pass: dP^T = V_j dO_i^T; dQ pass: dP = dO_i V_j^T
+        if constexpr (C::kTmemA) {
+            issue_ts_a(C::kColS, C::kColA0, st0);    // S = Q_i K_j^T, Q_i from TMEM
+            issue_ts_a(C::kColDP, C::kColA1, st1);   // dP = dO_i V_j^T, dO_i from TMEM
+        } else {
+            issue_ss(C::kColS, sFix0, st0);    // dK/dV pass: S^T = K_j Q_i^T;  dQ pass: S = Q_i K_j^T
+            issue_ss(C::kColDP, sFix1, st1);   // dK/dV pass: dP^T = V_j dO_i^T; dQ pass: dP = dO_i V_j^T
+        }
         tc_commit_if(leader, bar(kBbSFull));
         return true;
     };
@@ -334,6 +354,17 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
         FA_TRACE_EV(KV ? 1 : 13, 21);
         ++fix_iter;
         tc_fence_after();
+        if constexpr (C::kTmemA) {
+            // Q_i and dO_i into TMEM (after the last unit's MMAs, which read the old copy, in
+            // issue order); their shared memory is released once the copies have completed.
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                tc_cp_128x256b_if(leader, tmem + C::kColA0 + 8u * (uint32_t)kk, make_sdesc_sw128(sFix0, 16, 1024) + off);
+                tc_cp_128x256b_if(leader, tmem + C::kColA1 + 8u * (uint32_t)kk, make_sdesc_sw128(sFix1, 16, 1024) + off);
+            }
+            tc_commit_if(leader, bar(kBbFixEmpty));
+        }
         if constexpr (C::kSep) {
             if (!issue_s_dp(pos)) { ok = false; break; }
         }
@@ -373,7 +404,7 @@ __device__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t bars, uint3
         }
         if (!ok) break;
         tc_commit_if(leader, bar(kBbAccFull));
-        tc_commit_if(leader, bar(kBbFixEmpty));
+        if constexpr (!C::kTmemA) tc_commit_if(leader, bar(kBbFixEmpty));
         ++acc_iter;
     }
     if (!ok) {

@@ -227,6 +227,16 @@ __device__ __forceinline__ void mma_ts_if(uint32_t leader, uint32_t d_tmem, uint
         "r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// Copy a 128-row x 256-bit block of a shared-memory matrix (described like an MMA operand) into
+// TMEM: row i to lane i, 8 consecutive 32-bit columns from taddr.  Asynchronous, issued by the
+// elected lane; ordered before later tcgen05.mma of the same thread, tracked by tcgen05.commit.
+__device__ __forceinline__ void tc_cp_128x256b_if(uint32_t leader, uint32_t taddr, uint64_t sdesc) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\tsetp.ne.b32 e, %0, 0;\n\t"
+        "@e tcgen05.cp.cta_group::1.128x256b [%1], %2;\n\t}" ::"r"(leader),
+        "r"(taddr), "l"(sdesc)
+        : "memory");
+}
 // D[tmem] (+)= A[smem desc] * B[smem desc]
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
