@@ -430,3 +430,21 @@ def test_paged_page_out_of_range_is_reported():
     fa.flex_attention(q.cuda(), kp.cuda(), vp.cuda(), bm, page_table=table.cuda())
     assert bm.device_status() == fa.FA_ERR_INVALID_ARG
     assert bm.device_status() == fa.FA_OK
+
+
+def test_paged_decode_full_size_every_row():
+    # The decode workload the bench times (B = 16, H = 16, one new token, contexts 1k-8k,
+    # shuffled 128-token pages), through the split path in the bench's launch configuration
+    # (chunks of several tiles each, so chunk boundaries fall inside a sequence), against the
+    # float64 oracle on every (b, h) row.
+    fa = fa_module()
+    dw = wl.DECODE_WORKLOADS[0]
+    q, k, v, kp, vp, table, lens = wl.make_decode(dw)
+    KV = k.shape[2]
+    bm = fa.create_block_mask(0, dw.B, None, dw.Q, KV, kv_lens=torch.from_numpy(lens).cuda())
+    out, lse = fa.flex_attention(q.cuda(), kp.cuda(), vp.cuda(), bm, page_table=table.cuda(), scale=dw.scale)
+    torch.cuda.synchronize()
+    assert bm.device_status() == fa.FA_OK
+    mm = oracle.make_mask_mod(0, kv_lens=lens)
+    O, L = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), mm, None, scale=dw.scale)
+    compare(out, lse, O, L)
