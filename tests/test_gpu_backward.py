@@ -219,3 +219,58 @@ def test_full_size_sampled_rows(w):
     _, rdk, rdv = _oracle(w, q, k, v, do, doc, rows=keys, b=b, h=h)
     _compare(dk[b:b + 1, h:h + 1], rdk, "dk rows", rows_sel=(0, 0, keys))
     _compare(dv[b:b + 1, h:h + 1], rdv, "dv rows", rows_sel=(0, 0, keys))
+
+
+def test_backward_with_per_batch_sequence_lengths():
+    # kv_lens masks keys past each batch element's own length (the mask's kv_lens); the
+    # backward reads the same lengths on its partial tiles.
+    fa = fa_module()
+    B, H, S, D = 2, 2, 700, 64
+    lens = np.array([700, 433], dtype=np.int32)
+    g = torch.Generator().manual_seed(61)
+    q, k, v, do = (torch.randn(B, H, S, D, generator=g).to(torch.bfloat16) for _ in range(4))
+    bm = fa.create_block_mask(C, B, None, S, S, kv_lens=torch.from_numpy(lens).cuda())
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    out, lse = fa.flex_attention(qd, kd, vd, bm)
+    dq, dk, dv = fa.flex_attention_backward(qd, kd, vd, out, lse, dod, bm)
+    torch.cuda.synchronize()
+    assert bm.device_status() == fa.FA_OK
+    mm = oracle.make_mask_mod(C, kv_lens=lens)
+    rdq, rdk, rdv = oracle.attention_backward(*(t.float().numpy() for t in (q, k, v, do)), mm)
+    _compare(dq, rdq, "dq")
+    _compare(dk, rdk, "dk")
+    _compare(dv, rdv, "dv")
+    # Keys past a batch element's length get no gradient at all.
+    assert not torch.any(dk[1, :, lens[1]:]) and not torch.any(dv[1, :, lens[1]:])
+
+
+@pytest.mark.parametrize("bs", [(256, 256), (128, 384)])
+def test_backward_from_kv_blocks_and_other_block_sizes(bs):
+    # The kernels work on 128-wide tiles whatever BLOCK_SIZE the lists are read back at, and a
+    # mask built from caller lists (BlockMask.from_kv_blocks) holds the same tiles: the
+    # gradients are bitwise those of the 128 x 128 mask.
+    fa = fa_module()
+    Q = KV = 1536
+    kind, window = C | SW, 700
+    w = wl.Workload("bwd_lists", B=1, H=2, S=Q, D=64, dtype="bf16", mask_kind=kind, window=window, seed=62)
+    q, k, v = (t.cuda() for t in wl.make_qkv(w))
+    do = wl.make_dout(w).cuda()
+    grads = []
+    ref = oracle.create_block_mask(oracle.make_mask_mod(kind, window=window), None, None, Q, KV, bs)
+    lists = [torch.from_numpy(np.ascontiguousarray(ref[n])).cuda()
+             for n in ("kv_num_blocks", "kv_indices", "full_kv_num_blocks", "full_kv_indices")]
+    masks = [fa.create_block_mask(kind, None, None, Q, KV, window=window),
+             fa.create_block_mask(kind, None, None, Q, KV, window=window, BLOCK_SIZE=bs),
+             fa.block_mask_from_kv_blocks(*lists, Q_LEN=Q, KV_LEN=KV, BLOCK_SIZE=bs, mask_kind=kind,
+                                          window=window)]
+    for bm in masks:
+        out, lse = fa.flex_attention(q, k, v, bm)
+        grads.append(fa.flex_attention_backward(q, k, v, out, lse, do, bm))
+        torch.cuda.synchronize()
+        assert bm.device_status() == fa.FA_OK
+    for g in grads[1:]:
+        assert all(torch.equal(a, b) for a, b in zip(g, grads[0]))
+    rdq, rdk, rdv = _oracle(w, *(t.cpu() for t in (q, k, v, do)))
+    _compare(grads[0][0], rdq, "dq")
+    _compare(grads[0][1], rdk, "dk")
+    _compare(grads[0][2], rdv, "dv")
