@@ -13,28 +13,33 @@
 // with lse the forward's log-sum-exp, so P is recomputed exactly as the forward formed it.
 //
 // Three kernels, all deterministic (no atomics, no order that depends on timing):
-//   bwd_preprocess_kernel   Delta per query row and lse in log2 units, into a caller-provided
-//                           workspace padded to whole 128-row blocks (+inf / 0 in the padding,
+//   bwd_preprocess_kernel   -Delta per query row and -lse in log2 units, into a caller-provided
+//                           workspace padded to whole 128-row blocks (-inf / 0 in the padding,
 //                           so padded rows get P = 0);
 //   dK/dV kernel            one unit per kv block j (kv-major lists of the mask): K_j, V_j stay
 //                           in shared memory while the query blocks i of the unit stream
 //                           through a ring of stages (Q_i, dO_i, lse_i, Delta_i);
 //                             S^T = K_j Q_i^T and dP^T = V_j dO_i^T     (SS MMAs into TMEM)
-//                             P^T, dS^T in registers, written back over S^T, dP^T as 16-bit
+//                             P^T, dS^T in registers, written back to TMEM as 16-bit pairs
 //                             dV += P^T dO_i and dK += dS^T Q_i          (TS MMAs, A from TMEM)
 //   dQ kernel               one unit per query block i: Q_i, dO_i stay, K_j, V_j stream in the
 //                           mask's dQ write order (descending or ascending j);
-//                             S = Q_i K_j^T, dP = dO_i V_j^T, dS over dP, dQ += dS K_j.
+//                             S = Q_i K_j^T, dP = dO_i V_j^T, dS in its own columns,
+//                             dQ += dS K_j.
 // Each CTA owns its unit's accumulators in TMEM, so every sum runs in a fixed order.
 //
 // Organisation of both main kernels (one persistent CTA per SM, 12 warps, units handed out
 // at run time longest first, as in the forward):
 //   warp 0      TMA producer;   warp 1 MMA issuer (one elected lane);   warp 2 TMEM allocation;
-//   warps 4-11  element-wise math, one TMEM lane (row) per thread; warps 4-7 take columns
-//               0-63 of the 128 x 128 tile, warps 8-11 columns 64-127, and in the epilogue
-//               warps 4-7 / 8-11 write the two accumulators (dV / dK) or the two halves of dQ.
-// TMEM (512 columns): S at 0, dP at 128 (the 16-bit P and dS are written over their first 64
-// columns), accumulators at 256 and 256 + D.  All waits are bounded.
+//   warps 4-11  element-wise math, one TMEM lane (row) per thread, in two groups (warps 4-7,
+//               8-11) that split each tile's columns; in the epilogue they write the two
+//               accumulators (dV / dK) or the two halves of dQ.
+// TMEM (512 columns), three layouts (BCfg): the dK/dV pass at D = 64 and the dQ pass keep P
+// and dS in columns of their own after the accumulators, so the next entry's S and dP are
+// computed while the math warps work (at D = 64 the dQ pass also holds Q_i and dO_i as MMA A
+// operands); the dK/dV pass at D = 128, whose accumulators take 256 columns, works in
+// half-steps of 64 queries with two 128-column buffers of S^T / dP^T, P and dS written over
+// the columns just read.  All waits are bounded.
 #include <cfloat>
 
 #include <cuda_fp16.h>
