@@ -89,10 +89,11 @@ struct Cfg {
     // O0 O1 (64 each) = 512, so the next Q K^T can overwrite S while P is still being
     // computed.  At D = 128, P_t is written over the first 64 columns of S_t.
     static constexpr bool kSepP = (D == 64);
-    // Pairs (of 16 per 32-column chunk) whose 2^x runs on the FMA pipe in full tiles,
-    // to take load off the MUFU unit; worth it only when a score_mod already spends MUFU
-    // time (tanh), per measurement.
-    static constexpr int emu_pairs(int score) { return score != 0 ? 4 : 0; }
+    // Pairs (of every 16) whose 2^x runs on the FMA pipe in full tiles, to take load off the
+    // MUFU unit; worth it only when a score_mod already spends MUFU time (tanh), per
+    // measurement (32k soft-cap + ALiBi: 0 of 16 835, 1 832, 2 850, 3 845, 4 827 TFLOP/s; 8k
+    // causal without a score_mod: 0 674, 1 655, 2 665, 4 648).
+    static constexpr int emu_pairs(int score) { return score != 0 ? 2 : 0; }
     __device__ static constexpr uint32_t colS(int t) { return (uint32_t)t * 128u; }
     __device__ static constexpr uint32_t colP(int t) {
         return kSepP ? 256u + (uint32_t)t * 64u : (uint32_t)t * 128u;
