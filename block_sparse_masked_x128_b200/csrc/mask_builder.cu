@@ -30,7 +30,10 @@
 namespace fa {
 namespace {
 
-constexpr int kThreads = 128;  // == kBlock: one thread per query row when resolving a tile
+constexpr int kThreads = 128;
+// The classifier: one thread per kv block of a query block's row (in chunks), and 16 warps to
+// resolve the row's ambiguous tiles (a query block holding a document boundary can have dozens).
+constexpr int kClsThreads = 512;
 
 __global__ void __launch_bounds__(kThreads) doc_block_stats_kernel(const int32_t* __restrict__ doc,
                                                                   int len, int nblk, int bs,
@@ -97,43 +100,80 @@ __device__ int classify_fast(const MaskSpec& m, int i, int j) {
     return kAmbiguous;
 }
 
-// Element-by-element classification of one tile by one warp: lane l walks query rows l,
-// l + 32, ... across the tile's keys; the warp stops as soon as it has seen both an allowed
-// and a masked pair (a partial tile), so only dead and full tiles are read in full.
+// Element-by-element classification of one tile by one warp, in 32 x 32 sub-blocks: lane l
+// holds key k0 + cb + l (and its document id) and walks the sub-block's 32 query rows, whose
+// document ids it gets from the lane that loaded them (one shuffle per row, no memory access
+// in the inner loop).  The warp stops as soon as it has seen both an allowed and a masked pair
+// (a partial tile); row blocks are visited first, last, then the rest, so a tile whose mask
+// changes only at its last rows (a document boundary near a block edge) is decided early.
+// Only dead and full tiles are read in full.
 __device__ int resolve_tile_warp(const MaskSpec& m, int i, int j) {
-    long long lo, hi;
-    interval_bounds(m, lo, hi);
+    long long lo64, hi64;
+    interval_bounds(m, lo64, hi64);
+    // q - kv of in-range pairs fits in 32 bits (lengths are below 2^31): clamp the bounds.
+    const int lo = (int)max(lo64, (long long)INT_MIN), hi = (int)min(hi64, (long long)INT_MAX);
     const int lane = threadIdx.x & 31;
     const int q0 = i * m.BQ, k0 = j * m.BKV;
+    const bool has_doc = (m.kind & FA_MASK_DOCUMENT) != 0;
+    const int nrb = (m.BQ + 31) / 32, ncb = (m.BKV + 31) / 32;
+    // Document ids of this lane's rows and keys, fetched up front (independent loads) for
+    // tiles of up to 128 x 128; larger blocks fetch them per sub-block.
+    constexpr int kPre = 4;
+    int pre_q[kPre], pre_k[kPre];
+#pragma unroll
+    for (int c = 0; c < kPre; ++c) {
+        const int qr = q0 + 32 * c + lane, kv = k0 + 32 * c + lane;
+        pre_q[c] = (has_doc && c < nrb && 32 * c + lane < m.BQ && qr < m.Q_LEN) ? m.doc[qr] : 0;
+        pre_k[c] = (has_doc && c < ncb && 32 * c + lane < m.BKV && kv < m.KV_LEN) ? m.doc[kv] : 0;
+    }
     bool any = false, all = true;
-    for (int rb = 0; rb < m.BQ; rb += 32) {
-        const int q = q0 + rb + lane;
-        const bool q_row = rb + lane < m.BQ;
-        if (q_row) {
-            const bool q_in = q < m.Q_LEN;
-            const int dq = (q_in && m.doc) ? m.doc[q] : 0;
-            for (int c = 0; c < m.BKV; ++c) {
-                const int kv = k0 + c;
-                bool live = q_in && kv < m.KV_LEN;
-                if (live) {
-                    const long long d = (long long)q - kv;
-                    live = d >= lo && d <= hi;
-                    if (live && (m.kind & FA_MASK_DOCUMENT)) live = (m.doc[kv] == dq);
+    for (int t = 0; t < nrb; ++t) {
+        const int rbi = t == 0 ? 0 : (t == 1 ? nrb - 1 : t - 1);
+        const int rb = 32 * rbi;
+        const int qr = q0 + rb + lane;
+        int my_dq = 0;
+#pragma unroll
+        for (int c = 0; c < kPre; ++c)
+            if (rbi == c) my_dq = pre_q[c];
+        if (rbi >= kPre) my_dq = (has_doc && rb + lane < m.BQ && qr < m.Q_LEN) ? m.doc[qr] : 0;
+        const int nrows = min(32, m.BQ - rb);
+        for (int cbi = 0; cbi < ncb; ++cbi) {
+            const int cb = 32 * cbi;
+            const bool in_tile = cb + lane < m.BKV;          // lanes past the tile's keys sit out
+            const int kv = k0 + cb + lane;
+            const bool k_ok = in_tile && kv < m.KV_LEN;
+            int dk = 0;
+#pragma unroll
+            for (int c = 0; c < kPre; ++c)
+                if (cbi == c) dk = pre_k[c];
+            if (cbi >= kPre) dk = (has_doc && k_ok) ? m.doc[kv] : 0;
+            bool sub_any = false, sub_all = true;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const int dq = __shfl_sync(0xffffffffu, my_dq, r);
+                const int q = q0 + rb + r;
+                const int d = q - kv;
+                const bool live = k_ok && q < m.Q_LEN && d >= lo && d <= hi && (!has_doc || dk == dq);
+                if (r < nrows) {
+                    sub_any |= live;
+                    sub_all &= live;
                 }
-                any |= live;
-                all &= live;
             }
+            if (in_tile) {
+                any |= sub_any;
+                all &= sub_all;
+            }
+            const bool a = __any_sync(0xffffffffu, any);
+            const bool f = __all_sync(0xffffffffu, all);
+            if (a && !f) return kPartial;
         }
-        const bool a = __any_sync(0xffffffffu, any);
-        const bool f = __all_sync(0xffffffffu, all);
-        if (a && !f) return kPartial;
     }
     const bool a = __any_sync(0xffffffffu, any);
     const bool f = __all_sync(0xffffffffu, all);
     return !a ? kDead : (f ? kFull : kPartial);
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kClsThreads)
 classify_compact_kernel(MaskSpec m, int separate_full, int32_t* __restrict__ kv_num,
                         int32_t* __restrict__ kv_idx, int32_t* __restrict__ full_num,
                         int32_t* __restrict__ full_idx) {
@@ -142,16 +182,16 @@ classify_compact_kernel(MaskSpec m, int separate_full, int32_t* __restrict__ kv_
     // Per-batch context length: keys past it count as masked (the block grid stays KVB wide).
     if (m.kv_lens) m.KV_LEN = max(0, min(m.KV_LEN, m.kv_lens[bh / m.maskH]));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    __shared__ int s_cls[kThreads];
-    __shared__ int s_amb[kThreads];
+    __shared__ int s_cls[kClsThreads];
+    __shared__ int s_amb[kClsThreads];
     __shared__ int s_namb;
-    __shared__ int s_wp[kThreads / 32], s_wf[kThreads / 32];
+    __shared__ int s_wp[kClsThreads / 32], s_wf[kClsThreads / 32];
 
     const size_t row = (size_t)bh * m.QB + i;
     int32_t* my_kv = kv_idx + row * m.KVB;
     int32_t* my_full = full_idx + row * m.KVB;
     int np = 0, nf = 0;
-    for (int jb = 0; jb < m.KVB; jb += kThreads) {
+    for (int jb = 0; jb < m.KVB; jb += kClsThreads) {
         const int j = jb + tid;
         int cls = (j < m.KVB) ? classify_fast(m, i, j) : kDead;
         if (tid == 0) s_namb = 0;
@@ -160,7 +200,7 @@ classify_compact_kernel(MaskSpec m, int separate_full, int32_t* __restrict__ kv_
         s_cls[tid] = cls;
         __syncthreads();
         const int namb = s_namb;
-        for (int a = warp; a < namb; a += kThreads / 32) {   // one warp per ambiguous tile
+        for (int a = warp; a < namb; a += kClsThreads / 32) {   // one warp per ambiguous tile
             const int t = s_amb[a];
             const int c = resolve_tile_warp(m, i, jb + t);
             if (lane == 0) s_cls[t] = c;
@@ -176,7 +216,7 @@ classify_compact_kernel(MaskSpec m, int separate_full, int32_t* __restrict__ kv_
         }
         __syncthreads();
         int op = np, of = nf, tp = 0, tf = 0;
-        for (int w = 0; w < kThreads / 32; ++w) {
+        for (int w = 0; w < kClsThreads / 32; ++w) {
             if (w < warp) {
                 op += s_wp[w];
                 of += s_wf[w];
@@ -191,8 +231,8 @@ classify_compact_kernel(MaskSpec m, int separate_full, int32_t* __restrict__ kv_
         nf += tf;
         __syncthreads();
     }
-    for (int t = np + tid; t < m.KVB; t += kThreads) my_kv[t] = 0;
-    for (int t = nf + tid; t < m.KVB; t += kThreads) my_full[t] = 0;
+    for (int t = np + tid; t < m.KVB; t += kClsThreads) my_kv[t] = 0;
+    for (int t = nf + tid; t < m.KVB; t += kClsThreads) my_full[t] = 0;
     if (tid == 0) {
         kv_num[row] = np;
         full_num[row] = nf;
@@ -580,7 +620,7 @@ cudaError_t launch_mask_lists(const MaskSpec& spec, int separate_full, int maskB
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    classify_compact_kernel<<<dim3(spec.QB, maskBH), kThreads, 0, stream>>>(
+    classify_compact_kernel<<<dim3(spec.QB, maskBH), kClsThreads, 0, stream>>>(
         s, separate_full, kv_num, kv_idx, full_num, full_idx);
     return cudaGetLastError();
 }
