@@ -353,15 +353,21 @@ def time_forward(w: wl.Workload, steps: int, warmup: int, world: int, rank: int,
     doc_d = torch.from_numpy(doc).to(dev) if doc is not None else None
     stream = torch.cuda.current_stream()
 
+    # Mask build: CUDA events around the whole call (its one device allocation, the copies and
+    # the kernels), every mask kept alive until all are timed so that no free (which
+    # synchronises the device) falls inside a timed build.
     build_ms = []
-    bm = None
+    masks = []
     for _ in range(5):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
         e0.record(stream)
-        bm = fa.create_block_mask(w.mask_kind, None, None, w.S, w.S, window=w.window, doc_id=doc_d)
+        masks.append(fa.create_block_mask(w.mask_kind, None, None, w.S, w.S, window=w.window, doc_id=doc_d))
         e1.record(stream)
         torch.cuda.synchronize()
         build_ms.append(e0.elapsed_time(e1))
+    bm = masks.pop()
+    del masks
     out = torch.empty_like(qd)
     lse = torch.empty(w.B, w.H, w.S, device=dev, dtype=torch.float32)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
