@@ -748,7 +748,8 @@ def run_reference(args, w: wl.Workload, world: int, rank: int) -> dict:
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "impl": "reference", "config": config_dict(w, world),
+            "data": "synthetic", "impl": "reference",
+            "config": dict(config_dict(w, world), l2="host cores: the float64 oracle, no GPU cache involved"),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"{tot_rows} query rows of {w.name} in {rows}-row chunks, about {per_step:.2g} s per step"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
