@@ -102,11 +102,13 @@ fa_status_t make_tmap(CUtensorMap* map, const fa_tensor_t* t, const char* name) 
 
 fa_status_t check_tensor(const fa_tensor_t* t, const char* name) {
     if (!t) return fail(FA_ERR_INVALID_ARG, "%s is NULL", name);
-    if (!t->data) return fail(FA_ERR_INVALID_ARG, "%s.data is NULL", name);
     if (t->dtype != FA_DTYPE_F16 && t->dtype != FA_DTYPE_BF16)
         return fail(FA_ERR_INVALID_ARG, "%s.dtype %d is not FA_DTYPE_F16/BF16", name, t->dtype);
     if (t->B < 0 || t->H < 0 || t->S < 0 || t->D <= 0)
         return fail(FA_ERR_INVALID_ARG, "%s has a negative or zero extent", name);
+    // An empty tensor (B, H or S of 0) may have no storage; nothing ever reads it.
+    if (!t->data && t->B != 0 && t->H != 0 && t->S != 0)
+        return fail(FA_ERR_INVALID_ARG, "%s.data is NULL", name);
     if (t->stride[3] != 1) return fail(FA_ERR_INVALID_ARG, "%s.stride[3] must be 1", name);
     for (int i = 0; i < 3; ++i)
         if (t->stride[i] <= 0 || (t->stride[i] % 8) != 0)
@@ -737,7 +739,8 @@ fa_status_t fa_backward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_ten
     if (score_mod_kind & ~known) return fail(FA_ERR_INVALID_ARG, "unknown score_mod_kind bits 0x%x", score_mod_kind);
     if ((score_mod_kind & FA_SCORE_SOFTCAP) && (!params || !(params->softcap > 0.f)))
         return fail(FA_ERR_INVALID_ARG, "soft-cap needs params->softcap > 0");
-    if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    const bool empty = q->B == 0 || q->H == 0 || q->S == 0 || k->S == 0;   // nothing to compute
+    if ((!lse && !empty) || (reinterpret_cast<uintptr_t>(lse) & 3u))
         return fail(FA_ERR_INVALID_ARG, "lse must be a 4-byte aligned device pointer");
     if (!m) return fail(FA_ERR_INVALID_ARG, "block_mask is NULL");
     if (q->S != m->Q_LEN || k->S != m->KV_LEN)
@@ -747,10 +750,10 @@ fa_status_t fa_backward(const fa_tensor_t* q, const fa_tensor_t* k, const fa_ten
         return fail(FA_ERR_INVALID_ARG, "mask B/H (%d, %d) neither broadcast nor equal to q's", m->B, m->H);
     if ((int64_t)(m->QB > m->KVB ? m->QB : m->KVB) * q->B * q->H > 0x7fffffffLL)
         return fail(FA_ERR_UNSUPPORTED, "too many work units");
+    if (empty) return ok();
     const size_t need = fa_backward_workspace_bytes(q->B, q->H, q->S);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15u))
         return fail(FA_ERR_INVALID_ARG, "workspace must be 16-byte aligned device memory of at least %zu bytes", need);
-    if (q->B == 0 || q->H == 0 || q->S == 0) return ok();
 
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

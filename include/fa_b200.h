@@ -99,7 +99,9 @@ typedef struct fa_score_params {
 /* A (B, H, S, D) tensor: batch, heads, sequence, head_dim, the layout shared with
  * scaled_dot_product_attention ("How to Use FlexAttention on Apple Silicon", Setup). */
 typedef struct fa_tensor {
-    void*   data;        /* device pointer, 16-byte aligned                         */
+    void*   data;        /* device pointer, 16-byte aligned; may be NULL when B, H or S is 0
+                            (an empty tensor: every call on empty operands does nothing
+                            and returns FA_OK)                                       */
     int32_t dtype;       /* FA_DTYPE_F16 or FA_DTYPE_BF16                           */
     int64_t B, H, S, D;
     int64_t stride[4];   /* element strides of B, H, S, D; stride[3] must be 1 and the

@@ -448,3 +448,33 @@ def test_paged_decode_full_size_every_row():
     mm = oracle.make_mask_mod(0, kv_lens=lens)
     O, L = oracle.attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), mm, None, scale=dw.scale)
     compare(out, lse, O, L)
+
+
+def test_empty_batches_and_unsupported_head_sizes():
+    # Degenerate shapes: an empty batch (B = 0) or no heads is a no-op for the forward, the
+    # backward, the masked softmax and the paged decode (nothing launched, status OK); head
+    # sizes other than 64 and 128 are refused before any launch; the context stays usable.
+    fa = fa_module()
+    bm = gpu_block_mask(C, None, None, 256, 256)
+    for shape in ((0, 2, 256, 64), (1, 0, 256, 64)):
+        q = torch.zeros(shape, dtype=torch.bfloat16, device="cuda")
+        out, lse = fa.flex_attention(q, q, q, bm)
+        dq, dk, dv = fa.flex_attention_backward(q, q, q, out, lse, q, bm)
+        torch.cuda.synchronize()
+        assert out.shape == q.shape and lse.shape == q.shape[:3] and dq.shape == q.shape
+        s = torch.zeros(shape[0], shape[1], 256, 256, dtype=torch.bfloat16, device="cuda")
+        assert fa.masked_softmax(s).shape == s.shape
+    assert bm.device_status() == fa.FA_OK
+    for D in (32, 96, 256):
+        q = torch.zeros(1, 1, 256, D, dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(fa.FaError) as info:
+            fa.flex_attention(q, q, q, bm)
+        assert info.value.status == fa.FA_ERR_UNSUPPORTED
+    # A one-row query against one key (the smallest live problem) still matches the oracle.
+    g = torch.Generator().manual_seed(27)
+    q, k, v = (torch.randn(1, 1, 1, 64, generator=g).to(torch.bfloat16) for _ in range(3))
+    bm1 = gpu_block_mask(C, None, None, 1, 1)
+    out, lse = fa.flex_attention(q.cuda(), k.cuda(), v.cuda(), bm1)
+    torch.cuda.synchronize()
+    assert torch.equal(out.cpu(), v)         # one key: O = V exactly
+    assert bm1.device_status() == fa.FA_OK
