@@ -20,6 +20,7 @@ namespace fa {
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr uint32_t kProducerSleepNs = 256;         // the producer's pause between polls
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;         // log2 of the largest P allowed
@@ -155,8 +156,11 @@ __device__ void producer_role(const FwdParams& p, const CUtensorMap* tmq, const 
                               volatile int* ring, volatile int* abort_flag) {
     const uint32_t sQ = sbase, sKV = sbase + 2 * C::kTileBytes;
     auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+    // The producer runs ahead of the MMA and softmax warps and mostly waits for a free stage;
+    // it sleeps between polls, so it takes fewer issue slots from the softmax warps that share
+    // its SM sub-partition (measured: +0.5 % at 8k and 32k, for 64 to 1024 ns alike).
     auto wait = [&](int i, uint32_t par) {
-        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
+        return mbar_wait_bounded_sleepy(bar(i), par, abort_flag, p.status, kWaitLimitNs, kProducerSleepNs);
     };
     const uint32_t leader = elect_one_lane();
     if (leader) {

@@ -100,6 +100,30 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     return __all_sync(kFullMask, ok);
 }
 
+// mbar_wait_bounded for a warp off the critical path: it sleeps `sleep_ns` between polls, so
+// its polling takes fewer issue slots from the warps that share its SM sub-partition.
+__device__ __forceinline__ bool mbar_wait_bounded_sleepy(uint32_t bar, uint32_t parity,
+                                                         volatile int* abort_flag, int* status,
+                                                         uint64_t limit_ns, uint32_t sleep_ns) {
+    bool ok = mbar_try_wait(bar, parity);
+    if (!ok) {
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t it = 1;; ++it) {
+            __nanosleep(sleep_ns);
+            if (mbar_try_wait(bar, parity)) { ok = true; break; }
+            if ((it & 15u) == 0u) {
+                if (*abort_flag) break;
+                if (global_timer_ns() - t0 > limit_ns) {
+                    *abort_flag = 1;
+                    atomicExch(status, 1);
+                    break;
+                }
+            }
+        }
+    }
+    return __all_sync(kFullMask, ok);
+}
+
 // 1 in exactly one lane of the (fully active) calling warp, 0 elsewhere.
 __device__ __forceinline__ uint32_t elect_one_lane() {
     uint32_t is_elected;
