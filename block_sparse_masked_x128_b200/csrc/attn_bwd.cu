@@ -175,8 +175,9 @@ __device__ void bwd_producer(const BwdParams& p, const CUtensorMap* tq, const CU
                              uint32_t bars, volatile int* ring, volatile int* abort_flag) {
     using C = BCfg<D, KV>;
     auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+    // Off the critical path (it runs ahead of the MMA warp): sleep between polls.
     auto wait = [&](int i, uint32_t par) {
-        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
+        return mbar_wait_bounded_sleepy(bar(i), par, abort_flag, p.status, kWaitLimitNs, kProducerSleepNs);
     };
     const CUtensorMap* fix0 = KV ? tk : tq;
     const CUtensorMap* fix1 = KV ? tv : tdo;
