@@ -204,25 +204,37 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
             tc_commit_if(leader, bar(C::kBarSlotEmpty + s));
             if (un.E == 1) tc_commit_if(leader, bar(kBarQEmpty));
         }
+        // Stage waits: V of entry e at position kbase + 2e + 1 and K of entry e + 1 right after it.
+        auto wait_slots = [&](uint32_t vp, bool with_k) -> bool {
+            if (!wait(C::kBarSlotFull + (int)(vp % C::kStages), (vp / C::kStages) & 1u)) return false;
+            const uint32_t kp = vp + 1u;
+            return !with_k || wait(C::kBarSlotFull + (int)(kp % C::kStages), (kp / C::kStages) & 1u);
+        };
+        bool slots_ready = false;   // this entry's stages were waited for during the last one
         for (int e = 0; e < un.E; ++e) {
             const bool has_next = e + 1 < un.E;
             const int next = has_next ? er.get(e + 1) : 0;
             const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u, kpos = vpos + 1u;
             const int vs = (int)(vpos % C::kStages), ks = (int)(kpos % C::kStages);
             FA_TRACE_EV(1, 22);
-            if (!wait(C::kBarSlotFull + vs, (vpos / C::kStages) & 1u)) { ok = false; break; }
-            if (has_next && !wait(C::kBarSlotFull + ks, (kpos / C::kStages) & 1u)) { ok = false; break; }
+            if (!slots_ready && !wait_slots(vpos, has_next)) { ok = false; break; }
             FA_TRACE_EV(1, 23);
             tc_fence_after();
             if constexpr (C::kSepP) {
                 // Per tile: the next S first (it only needs the softmax to have read the
                 // current S), then P.V of the current entry.  Tile 0 runs ahead of tile 1
-                // (the softmax groups take turns), so tile 0 is served first.
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    if (ok && (next & (t ? kLive1 : kLive0))) ok = do_qk(t, ks);
-                    if (ok && (code & (t ? kLive1 : kLive0))) ok = do_pv(t, vs);
+                // (the softmax groups take turns), so tile 0 is served first.  The next
+                // entry's stages are waited for while tile 1's P is still being computed, so
+                // that wait stays off the path from tile 1's P to tile 0's next S.
+                if (ok && (next & kLive0)) ok = do_qk(0, ks);
+                if (ok && (code & kLive0)) ok = do_pv(0, vs);
+                if (ok && (next & kLive1)) ok = do_qk(1, ks);
+                slots_ready = false;
+                if (ok && has_next) {
+                    ok = wait_slots(vpos + 2u, e + 2 < un.E);
+                    slots_ready = true;
                 }
+                if (ok && (code & kLive1)) ok = do_pv(1, vs);
             } else {
                 // P_t lives in S_t: P.V of the current entry must be issued before the
                 // next Q K^T overwrites it.
