@@ -19,7 +19,9 @@
 // A work unit is a pair of adjacent query blocks (2p, 2p+1) of one (b, h); both tiles
 // share every K/V load of the merged kv-block list.  The MMA warp serves tile 0, then
 // tile 1, for every entry; that fixed order keeps the two softmax groups about half a
-// tile apart, so one group's exponentials run while the other waits for its next S.
+// tile apart, so one group's exponentials run while the other waits for its next S.  At
+// D = 64 tile 0's Q K^T runs one entry further ahead than tile 1's (its next S is computed
+// before tile 1's P.V), so it is ready when tile 0's softmax needs it.
 //
 // TMEM (512 columns x 128 lanes, fp32):
 //   D = 64:  S0 at 0, S1 at 128, P0 at 256, P1 at 320 (16-bit pairs), O0 at 384, O1 at 448;
@@ -191,66 +193,89 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
         };
         EntryReader er;
         er.init(un.entries, un.E);
+        // Stage of ring position pos, and the wait for its TMA load; K of entry e sits at
+        // kbase + 2e and V of entry e right after it.
+        auto stage = [&](uint32_t pos) { return (int)(pos % C::kStages); };
+        auto wait_pos = [&](uint32_t pos) {
+            return wait(C::kBarSlotFull + stage(pos), (pos / C::kStages) & 1u);
+        };
         int code = er.get(0);
         {   // S for entry 0
-            const uint32_t pos = kbase;
-            const int s = (int)(pos % C::kStages);
-            if (!wait(C::kBarSlotFull + s, (pos / C::kStages) & 1u)) { ok = false; break; }
+            if (!wait_pos(kbase)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int t = 0; t < 2; ++t)
-                if (ok && (code & (t ? kLive1 : kLive0))) ok = do_qk(t, s);
+                if (ok && (code & (t ? kLive1 : kLive0))) ok = do_qk(t, stage(kbase));
             if (!ok) break;
-            tc_commit_if(leader, bar(C::kBarSlotEmpty + s));
+            tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(kbase)));
             if (un.E == 1) tc_commit_if(leader, bar(kBarQEmpty));
         }
-        // Stage waits: V of entry e at position kbase + 2e + 1 and K of entry e + 1 right after it.
-        auto wait_slots = [&](uint32_t vp, bool with_k) -> bool {
-            if (!wait(C::kBarSlotFull + (int)(vp % C::kStages), (vp / C::kStages) & 1u)) return false;
-            const uint32_t kp = vp + 1u;
-            return !with_k || wait(C::kBarSlotFull + (int)(kp % C::kStages), (kp / C::kStages) & 1u);
-        };
-        bool slots_ready = false;   // this entry's stages were waited for during the last one
-        for (int e = 0; e < un.E; ++e) {
-            const bool has_next = e + 1 < un.E;
-            const int next = has_next ? er.get(e + 1) : 0;
-            const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u, kpos = vpos + 1u;
-            const int vs = (int)(vpos % C::kStages), ks = (int)(kpos % C::kStages);
-            FA_TRACE_EV(1, 22);
-            if (!slots_ready && !wait_slots(vpos, has_next)) { ok = false; break; }
-            FA_TRACE_EV(1, 23);
-            tc_fence_after();
-            if constexpr (C::kSepP) {
-                // Per tile: the next S first (it only needs the softmax to have read the
-                // current S), then P.V of the current entry.  Tile 0 runs ahead of tile 1
-                // (the softmax groups take turns), so tile 0 is served first.  The next
-                // entry's stages are waited for while tile 1's P is still being computed, so
-                // that wait stays off the path from tile 1's P to tile 0's next S.
-                if (ok && (next & kLive0)) ok = do_qk(0, ks);
-                if (ok && (code & kLive0)) ok = do_pv(0, vs);
-                if (ok && (next & kLive1)) ok = do_qk(1, ks);
-                slots_ready = false;
-                if (ok && has_next) {
-                    ok = wait_slots(vpos + 2u, e + 2 < un.E);
-                    slots_ready = true;
+        if constexpr (C::kSepP) {
+            // Tile 0's Q K^T runs one entry further ahead than tile 1's.  Per entry e the
+            // stream is: P.V of tile 0 (e), S of tile 1 (e + 1), S of tile 0 (e + 2), P.V of
+            // tile 1 (e).  A tile's next S only needs its softmax to hold the current S in
+            // registers, which tile 0's does about half a period before tile 1 publishes P,
+            // so tile 0's next S is ready when its softmax finishes the current one.
+            int next = un.E > 1 ? er.get(1) : 0;
+            if (un.E > 1) {   // S of tile 0 for entry 1
+                if (!wait_pos(kbase + 2u)) { ok = false; break; }
+                tc_fence_after();
+                if (next & kLive0) ok = do_qk(0, stage(kbase + 2u));
+                if (!ok) break;
+            }
+            for (int e = 0; e < un.E; ++e) {
+                const bool has1 = e + 1 < un.E, has2 = e + 2 < un.E;
+                const int next2 = has2 ? er.get(e + 2) : 0;
+                const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u;   // V(e); K(e + 1) follows
+                FA_TRACE_EV(1, 22);
+                if (!wait_pos(vpos)) { ok = false; break; }
+                FA_TRACE_EV(1, 23);
+                tc_fence_after();
+                if (code & kLive0) ok = do_pv(0, stage(vpos));
+                if (ok && has1 && (next & kLive1)) ok = do_qk(1, stage(vpos + 1u));
+                if (ok && has2) {
+                    if (!wait_pos(vpos + 3u)) {   // K(e + 2)
+                        ok = false;
+                    } else {
+                        tc_fence_after();
+                        if (next2 & kLive0) ok = do_qk(0, stage(vpos + 3u));
+                    }
                 }
-                if (ok && (code & kLive1)) ok = do_pv(1, vs);
-            } else {
+                if (ok && (code & kLive1)) ok = do_pv(1, stage(vpos));
+                if (!ok) break;
+                tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(vpos)));
+                if (has1) {   // both tiles' S of entry e + 1 are issued
+                    tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(vpos + 1u)));
+                    if (e + 2 == un.E) tc_commit_if(leader, bar(kBarQEmpty));
+                }
+                code = next;
+                next = next2;
+            }
+        } else {
+            for (int e = 0; e < un.E; ++e) {
+                const bool has_next = e + 1 < un.E;
+                const int next = has_next ? er.get(e + 1) : 0;
+                const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u, kpos = vpos + 1u;
+                FA_TRACE_EV(1, 22);
+                if (!wait_pos(vpos)) { ok = false; break; }
+                if (has_next && !wait_pos(kpos)) { ok = false; break; }
+                FA_TRACE_EV(1, 23);
+                tc_fence_after();
                 // P_t lives in S_t: P.V of the current entry must be issued before the
                 // next Q K^T overwrites it.
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
-                    if (ok && (code & (t ? kLive1 : kLive0))) ok = do_pv(t, vs);
-                    if (ok && (next & (t ? kLive1 : kLive0))) ok = do_qk(t, ks);
+                    if (ok && (code & (t ? kLive1 : kLive0))) ok = do_pv(t, stage(vpos));
+                    if (ok && (next & (t ? kLive1 : kLive0))) ok = do_qk(t, stage(kpos));
                 }
+                if (!ok) break;
+                tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(vpos)));
+                if (has_next) {
+                    tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(kpos)));
+                    if (e + 2 == un.E) tc_commit_if(leader, bar(kBarQEmpty));
+                }
+                code = next;
             }
-            if (!ok) break;
-            tc_commit_if(leader, bar(C::kBarSlotEmpty + vs));
-            if (has_next) {
-                tc_commit_if(leader, bar(C::kBarSlotEmpty + ks));
-                if (e + 2 == un.E) tc_commit_if(leader, bar(kBarQEmpty));
-            }
-            code = next;
         }
         if (!ok) break;
 #pragma unroll
