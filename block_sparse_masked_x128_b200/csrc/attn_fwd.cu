@@ -12,16 +12,17 @@
 //               the unit's Q tiles and K_j, V_j of every listed kv block into a ring of
 //               shared-memory stages (128-byte swizzle).
 //   warp 1      MMA issuer (one elected lane): S_t = Q_t K_j^T into TMEM (SS MMA), and
-//               O_t += P_t V_j with P_t read from TMEM (TS MMA).
-//   warp 2      TMEM allocation / release; warp 3 idle (completes the warpgroup).
+//               O_t += P_t V_j with P_t read from TMEM (TS MMA); at D = 64 for tile 0 only,
+//               at D = 128 for both tiles.
+//   warp 2      TMEM allocation / release.
+//   warp 3      at D = 64 the MMA issuer of tile 1; idle at D = 128 (completes the warpgroup).
 //   warps 4-7   softmax for query tile 0 (one thread per query row = TMEM lane),
 //   warps 8-11  softmax for query tile 1.
 // A work unit is a pair of adjacent query blocks (2p, 2p+1) of one (b, h); both tiles
-// share every K/V load of the merged kv-block list.  The MMA warp serves tile 0, then
-// tile 1, for every entry; that fixed order keeps the two softmax groups about half a
+// share every K/V load of the merged kv-block list.  At D = 128 one MMA warp serves tile 0,
+// then tile 1, for every entry; that fixed order keeps the two softmax groups about half a
 // tile apart, so one group's exponentials run while the other waits for its next S.  At
-// D = 64 tile 0's Q K^T runs one entry further ahead than tile 1's (its next S is computed
-// before tile 1's P.V), so it is ready when tile 0's softmax needs it.
+// D = 64 each tile has its own MMA warp, whose stream waits only on that tile's softmax.
 //
 // TMEM (512 columns x 128 lanes, fp32):
 //   D = 64:  S0 at 0, S1 at 128, P0 at 256, P1 at 320 (16-bit pairs), O0 at 384, O1 at 448;
@@ -68,10 +69,10 @@ enum : int {
     kBarOFree = 8,    // + tile
     kBarSFree = 10,   // + tile: softmax has S in registers (separate-P layout only)
     kBarPVDone = 12,  // + tile: the tile's last P.V has completed (separate-P layout only)
-    kBarDrain = 14,
-    kBarUnitFull = 15,  // + unit-ring slot (2)
-    kBarUnitEmpty = 17, // + unit-ring slot (2)
-    kBarSlotBase = 19   // + stage, then slot-empty barriers follow
+    kBarDrain = 14,     // + tile
+    kBarUnitFull = 16,  // + unit-ring slot (2)
+    kBarUnitEmpty = 18, // + unit-ring slot (2)
+    kBarSlotBase = 20   // + stage, then slot-empty barriers follow
 };
 
 template <int D>
@@ -91,6 +92,8 @@ struct Cfg {
     // O0 O1 (64 each) = 512, so the next Q K^T can overwrite S while P is still being
     // computed.  At D = 128, P_t is written over the first 64 columns of S_t.
     static constexpr bool kSepP = (D == 64);
+    // MMA warps: one per query tile with separate P (warps 1 and 3), else warp 1 for both.
+    static constexpr int kMmaWarps = kSepP ? 2 : 1;
     // Pairs (of every 16) whose 2^x runs on the FMA pipe in full tiles, to take load off the
     // MUFU unit; worth it only when a score_mod already spends MUFU time (tanh), per
     // measurement (32k soft-cap + ALiBi: 0 of 16 835, 1 832, 2 850, 3 845, 4 827 TFLOP/s; 8k
@@ -105,25 +108,19 @@ struct Cfg {
     }
 };
 
-// ------------------------------------------------------------------ MMA issuer (warp 1)
+// ------------------------------------------------------------------ MMA issuers (warps 1, 3)
 
+// The tensor-core work of one query tile t, issued by the elected lane of the calling warp.
 template <int D, bool BF16>
-__device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
-                         const volatile int* ring, volatile int* abort_flag) {
+struct TileMma {
     using C = Cfg<D>;
-    const uint32_t leader = elect_one_lane();
-    const uint32_t sQ = sbase, sKV = sbase + 2 * C::kTileBytes;
-    constexpr uint32_t kIdescQK = make_idesc_f16(BF16, 128, 128, false);
-    constexpr uint32_t kIdescPV = make_idesc_f16(BF16, 128, D, true);
-    auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
-    auto wait = [&](int i, uint32_t par) {
-        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
-    };
+    uint32_t leader, sQ, sKV, tmem;
     // S_t = Q_t K^T: M = 128 query rows, N = 128 keys, K = D in steps of 16.  Both
     // operands are K-major with 128-byte swizzle: 8-row atoms 1024 bytes apart (SBO),
     // a step of 16 elements is 32 bytes inside the atom, and columns 64.. live in the
     // next 16 KB box.
-    auto issue_qk = [&](int t, int slot) {
+    __device__ __forceinline__ void qk(int t, int slot) const {
+        constexpr uint32_t kIdescQK = make_idesc_f16(BF16, 128, 128, false);
         const uint32_t d = tmem + C::colS(t);
         const uint64_t qd = make_sdesc_sw128(sQ + t * C::kTileBytes, 16, 1024);
         const uint64_t kd = make_sdesc_sw128(sKV + slot * C::kTileBytes, 16, 1024);
@@ -133,11 +130,12 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
             const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
             mma_ss_if(leader, d, qd + off, kd + off, kIdescQK, kk > 0 ? 1u : 0u);
         }
-    };
+    }
     // O_t += P_t V: M = 128, N = D, K = 128 keys in steps of 16.  P_t comes from TMEM
     // (8 columns of packed pairs per step).  V is MN-major (D contiguous): 16 keys are
     // two 8-row atoms (SBO = 1024 bytes), 64-column boxes 16 KB apart (LBO).
-    auto issue_pv = [&](int t, int slot, bool accumulate) {
+    __device__ __forceinline__ void pv(int t, int slot, bool accumulate) const {
+        constexpr uint32_t kIdescPV = make_idesc_f16(BF16, 128, D, true);
         const uint32_t d = tmem + C::colO(t);
         const uint32_t pa = tmem + C::colP(t);
         const uint64_t vd = make_sdesc_sw128(sKV + slot * C::kTileBytes, 16384, 1024);
@@ -146,23 +144,148 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
             mma_ts_if(leader, d, pa + (uint32_t)(kk * 8), vd + (uint64_t)((kk * 2048) >> 4), kIdescPV,
                       (kk > 0 || accumulate) ? 1u : 0u);
         }
-    };
+    }
+};
 
-    uint32_t kv_pos = 0, q_iter = 0;
-    uint32_t pf_cnt[2] = {0u, 0u}, of_cnt[2] = {0u, 0u}, qk_cnt[2] = {0u, 0u};
+// MMA issuer of one query tile t (the D = 64 layout, S and P apart in TMEM): warp 1 serves
+// tile 0 and warp 3 tile 1, so each tile's stream waits only on its own softmax group and the
+// issue work is split between two SM sub-partitions (686 -> 700 TFLOP/s at 8k causal).  Both
+// warps commit to each stage-empty and Q-empty barrier.
+template <int D, bool BF16>
+__device__ void mma_role_tile(const FwdParams& p, int t, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                              const volatile int* ring, volatile int* abort_flag) {
+    using C = Cfg<D>;
+    static_assert(C::kSepP, "one MMA warp per tile needs S and P apart");
+    TileMma<D, BF16> mma;
+    mma.leader = elect_one_lane();
+    mma.sQ = sbase;
+    mma.sKV = sbase + 2 * C::kTileBytes;
+    mma.tmem = tmem;
+    const uint32_t leader = mma.leader;
+    const int live = t ? kLive1 : kLive0;
+    const int tslot = t ? 10 : 1;   // trace slot of this warp
+    (void)tslot;
+    auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+    auto wait = [&](int i, uint32_t par) {
+        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
+    };
+    uint32_t kv_pos = 0, q_iter = 0, pf_cnt = 0, of_cnt = 0, qk_cnt = 0;
     bool ok = true;
     FA_TRACE_DECL
-    // S_t = Q_t K^T into TMEM; with separate P it first waits until the softmax holds the
-    // previous S_t in registers.
-    auto do_qk = [&](int t, int slot) -> bool {
-        if constexpr (C::kSepP) {
-            if (!wait(kBarSFree + t, (qk_cnt[t] & 1u) ^ 1u)) return false;
-            tc_fence_after();
-        }
-        ++qk_cnt[t];
-        issue_qk(t, slot);
+    // S_t = Q_t K^T into TMEM once the softmax holds the previous S_t in registers.
+    auto do_qk = [&](int slot) -> bool {
+        if (!wait(kBarSFree + t, (qk_cnt & 1u) ^ 1u)) return false;
+        tc_fence_after();
+        ++qk_cnt;
+        mma.qk(t, slot);
         tc_commit_if(leader, bar(kBarSFull + t));
         return true;
+    };
+    // Stage of ring position pos, and the wait for its TMA load; K of entry e sits at
+    // kbase + 2e and V of entry e right after it.
+    auto stage = [&](uint32_t pos) { return (int)(pos % C::kStages); };
+    auto wait_pos = [&](uint32_t pos) {
+        return wait(C::kBarSlotFull + stage(pos), (pos / C::kStages) & 1u);
+    };
+    uint32_t u_iter = 0;
+    for (;;) {
+        const int u = take_unit<C>(p, bars, ring, u_iter, abort_flag, ok);
+        if (u < 0) break;
+        const Unit un = decode_unit(p, u);
+        if (un.E == 0) continue;
+        const int nl = t ? un.nl1 : un.nl0;
+        if (!wait(kBarQFull, q_iter & 1u)) { ok = false; break; }
+        ++q_iter;
+        tc_fence_after();
+        const uint32_t kbase = kv_pos;
+        kv_pos += 2u * (uint32_t)un.E;
+        int ndone = 0;
+        // O_t += P_t V once the softmax has published P_t.
+        auto do_pv = [&](int slot) -> bool {
+            FA_TRACE_EV(tslot, 16 + t);
+            if (!wait(kBarPFull + t, pf_cnt & 1u)) return false;
+            FA_TRACE_EV(tslot, 18 + t);
+            ++pf_cnt;
+            if (ndone == 0 && !wait(kBarOFree + t, (of_cnt & 1u) ^ 1u)) return false;
+            tc_fence_after();
+            mma.pv(t, slot, ndone > 0);
+            tc_commit_if(leader, bar(kBarPVDone + t));
+            if (ndone + 1 == nl) tc_commit_if(leader, bar(kBarOFull + t));
+            ++ndone;
+            return true;
+        };
+        EntryReader er;
+        er.init(un.entries, un.E);
+        int code = er.get(0);
+        {   // S for entry 0
+            if (!wait_pos(kbase)) { ok = false; break; }
+            tc_fence_after();
+            if (code & live) ok = do_qk(stage(kbase));
+            if (!ok) break;
+            tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(kbase)));
+            if (un.E == 1) tc_commit_if(leader, bar(kBarQEmpty));
+        }
+        for (int e = 0; e < un.E; ++e) {
+            const bool has_next = e + 1 < un.E;
+            const int next = has_next ? er.get(e + 1) : 0;
+            const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u, kpos = vpos + 1u;
+            FA_TRACE_EV(tslot, 22);
+            if (!wait_pos(vpos)) { ok = false; break; }
+            if (has_next && !wait_pos(kpos)) { ok = false; break; }
+            FA_TRACE_EV(tslot, 23);
+            tc_fence_after();
+            // The next S first (it only needs the softmax to hold the current S), then P.V of
+            // the current entry.
+            if (next & live) ok = do_qk(stage(kpos));
+            if (ok && (code & live)) ok = do_pv(stage(vpos));
+            if (!ok) break;
+            tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(vpos)));
+            if (has_next) {
+                tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(kpos)));
+                if (e + 2 == un.E) tc_commit_if(leader, bar(kBarQEmpty));
+            }
+            code = next;
+        }
+        if (!ok) break;
+        if (nl > 0) ++of_cnt;
+    }
+    if (!ok) {
+        // Wait for every MMA this warp issued before the CTA can release TMEM.
+        tc_commit_if(leader, bar(kBarDrain + t));
+        drain_wait(bar(kBarDrain + t), 0u);
+    }
+}
+
+// MMA issuer of both query tiles (the D = 128 layout, P over S), warp 1: tile 0 then tile 1 for
+// every entry, P.V of the current entry before the next Q K^T (which overwrites P).  The fixed
+// order keeps the two softmax groups half a period apart; with one warp per tile they drift
+// into step (854 -> 718 TFLOP/s at 32k soft-cap, 718 -> 672 sliding window).
+template <int D, bool BF16>
+__device__ void mma_role_pair(const FwdParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                              const volatile int* ring, volatile int* abort_flag) {
+    using C = Cfg<D>;
+    static_assert(!C::kSepP, "the paired issuer is for P over S");
+    TileMma<D, BF16> mma;
+    mma.leader = elect_one_lane();
+    mma.sQ = sbase;
+    mma.sKV = sbase + 2 * C::kTileBytes;
+    mma.tmem = tmem;
+    const uint32_t leader = mma.leader;
+    auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+    auto wait = [&](int i, uint32_t par) {
+        return mbar_wait_bounded(bar(i), par, abort_flag, p.status, kWaitLimitNs);
+    };
+    uint32_t kv_pos = 0, q_iter = 0;
+    uint32_t pf_cnt[2] = {0u, 0u}, of_cnt[2] = {0u, 0u};
+    bool ok = true;
+    FA_TRACE_DECL
+    auto do_qk = [&](int t, int slot) {
+        mma.qk(t, slot);
+        tc_commit_if(leader, bar(kBarSFull + t));
+    };
+    auto stage = [&](uint32_t pos) { return (int)(pos % C::kStages); };
+    auto wait_pos = [&](uint32_t pos) {
+        return wait(C::kBarSlotFull + stage(pos), (pos / C::kStages) & 1u);
     };
     uint32_t u_iter = 0;
     for (;;) {
@@ -185,97 +308,44 @@ __device__ void mma_role(const FwdParams& p, uint32_t sbase, uint32_t bars, uint
             ++pf_cnt[t];
             if (ndone[t] == 0 && !wait(kBarOFree + t, (of_cnt[t] & 1u) ^ 1u)) return false;
             tc_fence_after();
-            issue_pv(t, slot, ndone[t] > 0);
-            if constexpr (C::kSepP) tc_commit_if(leader, bar(kBarPVDone + t));
+            mma.pv(t, slot, ndone[t] > 0);
             if (ndone[t] + 1 == nl[t]) tc_commit_if(leader, bar(kBarOFull + t));
             ++ndone[t];
             return true;
         };
         EntryReader er;
         er.init(un.entries, un.E);
-        // Stage of ring position pos, and the wait for its TMA load; K of entry e sits at
-        // kbase + 2e and V of entry e right after it.
-        auto stage = [&](uint32_t pos) { return (int)(pos % C::kStages); };
-        auto wait_pos = [&](uint32_t pos) {
-            return wait(C::kBarSlotFull + stage(pos), (pos / C::kStages) & 1u);
-        };
         int code = er.get(0);
         {   // S for entry 0
             if (!wait_pos(kbase)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int t = 0; t < 2; ++t)
-                if (ok && (code & (t ? kLive1 : kLive0))) ok = do_qk(t, stage(kbase));
-            if (!ok) break;
+                if (code & (t ? kLive1 : kLive0)) do_qk(t, stage(kbase));
             tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(kbase)));
             if (un.E == 1) tc_commit_if(leader, bar(kBarQEmpty));
         }
-        if constexpr (C::kSepP) {
-            // Tile 0's Q K^T runs one entry further ahead than tile 1's.  Per entry e the
-            // stream is: P.V of tile 0 (e), S of tile 1 (e + 1), S of tile 0 (e + 2), P.V of
-            // tile 1 (e).  A tile's next S only needs its softmax to hold the current S in
-            // registers, which tile 0's does about half a period before tile 1 publishes P,
-            // so tile 0's next S is ready when its softmax finishes the current one.
-            int next = un.E > 1 ? er.get(1) : 0;
-            if (un.E > 1) {   // S of tile 0 for entry 1
-                if (!wait_pos(kbase + 2u)) { ok = false; break; }
-                tc_fence_after();
-                if (next & kLive0) ok = do_qk(0, stage(kbase + 2u));
-                if (!ok) break;
-            }
-            for (int e = 0; e < un.E; ++e) {
-                const bool has1 = e + 1 < un.E, has2 = e + 2 < un.E;
-                const int next2 = has2 ? er.get(e + 2) : 0;
-                const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u;   // V(e); K(e + 1) follows
-                FA_TRACE_EV(1, 22);
-                if (!wait_pos(vpos)) { ok = false; break; }
-                FA_TRACE_EV(1, 23);
-                tc_fence_after();
-                if (code & kLive0) ok = do_pv(0, stage(vpos));
-                if (ok && has1 && (next & kLive1)) ok = do_qk(1, stage(vpos + 1u));
-                if (ok && has2) {
-                    if (!wait_pos(vpos + 3u)) {   // K(e + 2)
-                        ok = false;
-                    } else {
-                        tc_fence_after();
-                        if (next2 & kLive0) ok = do_qk(0, stage(vpos + 3u));
-                    }
-                }
-                if (ok && (code & kLive1)) ok = do_pv(1, stage(vpos));
-                if (!ok) break;
-                tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(vpos)));
-                if (has1) {   // both tiles' S of entry e + 1 are issued
-                    tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(vpos + 1u)));
-                    if (e + 2 == un.E) tc_commit_if(leader, bar(kBarQEmpty));
-                }
-                code = next;
-                next = next2;
-            }
-        } else {
-            for (int e = 0; e < un.E; ++e) {
-                const bool has_next = e + 1 < un.E;
-                const int next = has_next ? er.get(e + 1) : 0;
-                const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u, kpos = vpos + 1u;
-                FA_TRACE_EV(1, 22);
-                if (!wait_pos(vpos)) { ok = false; break; }
-                if (has_next && !wait_pos(kpos)) { ok = false; break; }
-                FA_TRACE_EV(1, 23);
-                tc_fence_after();
-                // P_t lives in S_t: P.V of the current entry must be issued before the
-                // next Q K^T overwrites it.
+        for (int e = 0; e < un.E; ++e) {
+            const bool has_next = e + 1 < un.E;
+            const int next = has_next ? er.get(e + 1) : 0;
+            const uint32_t vpos = kbase + 2u * (uint32_t)e + 1u, kpos = vpos + 1u;
+            FA_TRACE_EV(1, 22);
+            if (!wait_pos(vpos)) { ok = false; break; }
+            if (has_next && !wait_pos(kpos)) { ok = false; break; }
+            FA_TRACE_EV(1, 23);
+            tc_fence_after();
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    if (ok && (code & (t ? kLive1 : kLive0))) ok = do_pv(t, stage(vpos));
-                    if (ok && (next & (t ? kLive1 : kLive0))) ok = do_qk(t, stage(kpos));
-                }
-                if (!ok) break;
-                tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(vpos)));
-                if (has_next) {
-                    tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(kpos)));
-                    if (e + 2 == un.E) tc_commit_if(leader, bar(kBarQEmpty));
-                }
-                code = next;
+            for (int t = 0; t < 2; ++t) {
+                if (ok && (code & (t ? kLive1 : kLive0))) ok = do_pv(t, stage(vpos));
+                if (ok && (next & (t ? kLive1 : kLive0))) do_qk(t, stage(kpos));
             }
+            if (!ok) break;
+            tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(vpos)));
+            if (has_next) {
+                tc_commit_if(leader, bar(C::kBarSlotEmpty + stage(kpos)));
+                if (e + 2 == un.E) tc_commit_if(leader, bar(kBarQEmpty));
+            }
+            code = next;
         }
         if (!ok) break;
 #pragma unroll
@@ -605,7 +675,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
 
     if (threadIdx.x == 0) {
         mbar_init(bars + 8u * kBarQFull, 1);
-        mbar_init(bars + 8u * kBarQEmpty, 1);
+        mbar_init(bars + 8u * kBarQEmpty, C::kMmaWarps);   // one commit per MMA warp
         for (int t = 0; t < 2; ++t) {
             mbar_init(bars + 8u * (kBarSFull + t), 1);
             mbar_init(bars + 8u * (kBarPFull + t), 4);   // one arrival per softmax warp
@@ -615,13 +685,14 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
             mbar_init(bars + 8u * (kBarPVDone + t), 1);
         }
         mbar_init(bars + 8u * kBarDrain, 1);
+        mbar_init(bars + 8u * (kBarDrain + 1), 1);
         for (int r = 0; r < kUnitRing; ++r) {
             mbar_init(bars + 8u * (C::kBarUFull + r), 1);    // the TMA warp publishes
-            mbar_init(bars + 8u * (C::kBarUEmpty + r), 9);   // the MMA warp + 8 softmax warps
+            mbar_init(bars + 8u * (C::kBarUEmpty + r), C::kMmaWarps + 8);   // MMA + softmax warps
         }
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(bars + 8u * (C::kBarSlotFull + s), 1);
-            mbar_init(bars + 8u * (C::kBarSlotEmpty + s), 1);
+            mbar_init(bars + 8u * (C::kBarSlotEmpty + s), C::kMmaWarps);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -641,8 +712,11 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUt
         regs_dec<kRegsProducer>();
         if (warp == 0) {
             producer_role<Cfg<D>>(p, &tmq, &tmk, &tmv, sbase, bars, ring, abort_flag);
-        } else if (warp == 1) {
-            mma_role<D, BF16>(p, sbase, bars, tmem, ring, abort_flag);
+        } else if (warp == 1 || (C::kMmaWarps == 2 && warp == 3)) {
+            if constexpr (C::kMmaWarps == 2)
+                mma_role_tile<D, BF16>(p, warp == 3 ? 1 : 0, sbase, bars, tmem, ring, abort_flag);
+            else
+                mma_role_pair<D, BF16>(p, sbase, bars, tmem, ring, abort_flag);
         }
     } else {
         regs_inc<kRegsSoftmax>();
