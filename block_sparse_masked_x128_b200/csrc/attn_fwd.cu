@@ -96,9 +96,10 @@ struct Cfg {
     static constexpr int kMmaWarps = kSepP ? 2 : 1;
     // Pairs (of every 16) whose 2^x runs on the FMA pipe in full tiles, to take load off the
     // MUFU unit; worth it only when a score_mod already spends MUFU time (tanh), per
-    // measurement (32k soft-cap + ALiBi: 0 of 16 835, 1 832, 2 850, 3 845, 4 827 TFLOP/s; 8k
-    // causal without a score_mod: 0 674, 1 655, 2 665, 4 648).
-    static constexpr int emu_pairs(int score) { return score != 0 ? 2 : 0; }
+    // measurement (32k soft-cap + ALiBi, with 4 to 6 of 16 tanh pairs on the FMA pipe: 0 of 16
+    // 874-877, 1 891-902, 2 886-887 TFLOP/s; 8k causal without a score_mod: 0 674, 1 655,
+    // 2 665, 4 648).
+    static constexpr int emu_pairs(int score) { return score != 0 ? 1 : 0; }
     __device__ static constexpr uint32_t colS(int t) { return (uint32_t)t * 128u; }
     __device__ static constexpr uint32_t colP(int t) {
         return kSepP ? 256u + (uint32_t)t * 64u : (uint32_t)t * 128u;
@@ -405,6 +406,14 @@ constexpr int kVarDocument = 4;
 // bfloat16 value for caps up to 32 (e^-60 at cap 30), and a key the fixed base drives below
 // the float range weighs less than 2^-39 of that row's largest term.
 constexpr int kVarFixedMax = 8;
+// Largest |s / cap| for which the soft-cap's tanh is taken from its Taylor polynomial.
+constexpr float kTanhPolyBound = 0.2f;
+// Pairs (of every 16) whose tanh comes from the polynomial when the bound holds; the rest stay
+// on the MUFU unit, which balances the two pipes (a polynomial pair costs the FMA pipe about as
+// long as a tanh.approx pair costs the MUFU).  Measured at 32k soft-cap + ALiBi with one exp2
+// pair on the FMA pipe: 0 of 16 855, 4 891, 5 900, 6 895 TFLOP/s; all 16 (and two exp2 pairs)
+// 832.
+constexpr int kTanhPolyPairs = 5;
 
 template <int D, bool BF16, int VAR>
 __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t tmem,
@@ -505,25 +514,63 @@ __device__ void softmax_role(const FwdParams& p, int t, uint32_t bars, uint32_t 
                 // score_mod on every position of the tile, in log2 units; masked
                 // positions are set to -inf afterwards (the mask decides liveness).
                 const float2 inv2 = make_float2(p.inv_softcap_scale, p.inv_softcap_scale);
-                const float2 cap2 = make_float2(p.softcap_log2, p.softcap_log2);
                 const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
                 const float2 sl2 = make_float2(slope_log2, slope_log2);
                 const float2 two = make_float2(2.f, 2.f);
                 float2 pos = make_float2((float)(kv0 - q), (float)(kv0 - q + 1));
-#pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    float2 y;
-                    if constexpr (has_softcap) {
-                        const float2 a = __fmul2_rn(x[i], inv2);
-                        y = __fmul2_rn(cap2, make_float2(tanh_approx(a.x), tanh_approx(a.y)));
-                    } else {
-                        y = __fmul2_rn(x[i], sc2);
-                    }
+                auto bias = [&](float2 y) {
                     if constexpr (has_alibi) {
                         y = __ffma2_rn(sl2, pos, y);
                         pos = __fadd2_rn(pos, two);
                     }
-                    x[i] = y;
+                    return y;
+                };
+                if constexpr (has_softcap) {
+                    // cap tanh(s / cap).  If every |s / cap| of this warp's rows in the tile is
+                    // at most kTanhPolyBound, kTanhPolyPairs of every 16 pairs take tanh from its
+                    // odd Taylor polynomial through a^7 on the FMA pipe (the series alternates,
+                    // so the error is below the first omitted term, 62/2835 a^9: under 6e-8 of
+                    // tanh there) and the rest from the MUFU's tanh.approx; otherwise all of
+                    // them from tanh.approx.  The cap (log2 units) is folded into the
+                    // coefficients.
+                    float am0 = 0.f, am1 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 64; i += 2) {
+                        am0 = max3(am0, fabsf(x[i].x), fabsf(x[i].y));
+                        am1 = max3(am1, fabsf(x[i + 1].x), fabsf(x[i + 1].y));
+                    }
+                    const bool poly = __all_sync(kFullMask, fmaxf(am0, am1) * fabsf(p.inv_softcap_scale) <=
+                                                                kTanhPolyBound);
+                    const float cap = p.softcap_log2;
+                    if (poly) {
+                        const float2 k1 = make_float2(cap, cap);
+                        const float2 k3 = make_float2(cap * (-1.0f / 3.0f), cap * (-1.0f / 3.0f));
+                        const float2 k5 = make_float2(cap * (2.0f / 15.0f), cap * (2.0f / 15.0f));
+                        const float2 k7 = make_float2(cap * (-17.0f / 315.0f), cap * (-17.0f / 315.0f));
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) {
+                            const float2 a = __fmul2_rn(x[i], inv2);
+                            if ((i & 15) < kTanhPolyPairs) {
+                                const float2 a2 = __fmul2_rn(a, a);
+                                float2 t = __ffma2_rn(k7, a2, k5);
+                                t = __ffma2_rn(t, a2, k3);
+                                t = __ffma2_rn(t, a2, k1);
+                                x[i] = bias(__fmul2_rn(a, t));
+                            } else {
+                                x[i] = bias(__fmul2_rn(k1, make_float2(tanh_approx(a.x), tanh_approx(a.y))));
+                            }
+                        }
+                    } else {
+                        const float2 cap2 = make_float2(cap, cap);
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) {
+                            const float2 a = __fmul2_rn(x[i], inv2);
+                            x[i] = bias(__fmul2_rn(cap2, make_float2(tanh_approx(a.x), tanh_approx(a.y))));
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) x[i] = bias(__fmul2_rn(x[i], sc2));
                 }
             }
             if (!full) {

@@ -237,6 +237,22 @@ def test_score_mods(score_kind, D, dtype):
     compare(out, lse, O, L)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_softcap_polynomial_and_mufu_paths_in_one_tile(D):
+    # A warp takes tanh from its polynomial when every |s / cap| of its 32 rows in a tile is at
+    # most 0.2, else from tanh.approx.  At cap 30 unscaled N(0, 1) scores stay under the bound;
+    # query rows scaled by 4 in every other 32-row group push their warps past it, so both paths
+    # run side by side in every tile.
+    w = wl.Workload("softcap_mix", B=1, H=2, S=1024, D=D, dtype="bf16", mask_kind=C,
+                    score_kind=wl.SCORE_SOFTCAP | wl.SCORE_ALIBI, softcap=30.0, seed=29)
+    q, k, v = wl.make_qkv(w)
+    rows = (torch.arange(w.S) // 32) % 2 == 1
+    q[:, :, rows, :] *= 4
+    out, lse, _ = run_gpu(w, q, k, v)
+    O, L = run_oracle(w, q, k, v)
+    compare(out, lse, O, L)
+
+
 def test_explicit_alibi_slopes():
     fa = fa_module()
     w = wl.Workload("alibi_slopes", B=1, H=4, S=512, D=128, dtype="bf16", mask_kind=C,
