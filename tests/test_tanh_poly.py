@@ -67,7 +67,7 @@ def test_relative_error_over_the_bound():
     rel = np.abs(got / want - 1.0)
     # Truncation (first omitted term 62/2835 a^9) is below 6e-8 of tanh at the bound; the rest
     # is float32 rounding of a few operations.
-    assert rel.max() < 5e-7
+    assert rel.max() < 3e-7
     trunc = 62 / 2835 * bound ** 9 / np.tanh(bound)
     assert trunc < 6e-8
 
